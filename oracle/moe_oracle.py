@@ -1,0 +1,231 @@
+"""Plain, slow, fp64 CPU oracle of the Grok-1-style sparse MoE layer forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports or calls this
+module: only the tests, the smoke check and the benchmark's CPU-baseline leg
+do.  It shares no code with the CUDA path; both sides receive the same input
+bits from the ``synth`` generator.
+
+Source of every step: the page "How does Grok-1 use a mixture-of-experts
+design?" (n4n.ai).  Sections cited below:
+  [Arch]    "The high-level architecture"          (GrokMoELayer.forward)
+  [Routing] "Routing: top-2 without auxiliary loss" (grok_router_forward and
+            the capacity-factor paragraph after it)
+  [Expert]  "Expert implementation: SwiGLU at scale" (SwiGLUExpert,
+            FusedSwiGLUExpert)
+  [EP]      "Expert parallelism vs. tensor parallelism" (moe_layer_ep_forward:
+            each expert's output is scaled by its routing weight)
+  [Trade]   "Tradeoffs: when MoE wins and when it doesn't" (expert_batch_size)
+  [Dyn]     "Training dynamics: expert specialization" (utilization statistic)
+and the page "Let Grok spill the beans on Grok" (Medium), whose feature list
+states that the layer output is the weighted sum of the active experts'
+outputs.
+
+Readings taken where the pages leave a step open (each one is listed, with its
+reason, in the design notes of the repository):
+  * capacity = ceil(capacity_factor * T * top_k / E) evaluated in double in that
+    order; capacity_factor = +inf (or E/top_k) means no drop;
+  * overflow is dropped lowest-token-index-first: an assignment (t, e) is kept
+    iff fewer than `capacity` earlier tokens were routed to e;
+  * the softmax runs over the two selected logits only and is not renormalised
+    after a drop; a token whose two assignments are both dropped outputs 0;
+  * equal logits rank the lower expert index first;
+  * silu(z) = z * sigmoid(z);
+  * an optional per-expert logit bias is added to the logits before top-k.
+The method is exact (no approximation), so every function below is the plain
+definition, in float64, with numpy's matmul as the only library primitive.
+Parity unpinned: none (each function is pinned by tests/test_oracle_pins.py).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------
+# input decoding (storage format only)
+# ----------------------------------------------------------------------------
+def to_f64(a: np.ndarray) -> np.ndarray:
+    """Widen stored inputs to float64: uint16 arrays hold bf16 bit patterns."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# [Routing] router logits, top-2, softmax over the two selected logits
+# ----------------------------------------------------------------------------
+def router_logits(x, w_router, logit_bias=None) -> np.ndarray:
+    """logits[t, e] = sum_i x[t, i] * w_router[e, i]  (hidden @ W_r.T), [Routing].
+
+    w_router is stored [E, d] as on the page.  ``logit_bias`` (length E) is
+    added to every token's logits before top-k when given.
+    """
+    lg = to_f64(x) @ to_f64(w_router).T
+    if logit_bias is not None:
+        lg = lg + np.asarray(logit_bias, dtype=np.float64)[None, :]
+    return lg
+
+
+def top2_softmax(logits: np.ndarray, top_k: int = 2):
+    """Top-k experts per token ordered by logit, then softmax over the k values.
+
+    [Arch] / [Routing]: topk over the E logits, then softmax of the selected
+    values only.  Ordering: descending logit; equal logits keep the lower
+    expert index first (stable sort of the negated logits).
+    Returns idx int32 [T, k] and w float64 [T, k].
+    """
+    lg = np.asarray(logits, dtype=np.float64)
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :top_k]
+    sel = np.take_along_axis(lg, order, axis=1)
+    m = sel.max(axis=1, keepdims=True)
+    ex = np.exp(sel - m)
+    w = ex / ex.sum(axis=1, keepdims=True)
+    return order.astype(np.int32), w
+
+
+def near_tie_gap(logits: np.ndarray, top_k: int = 2) -> np.ndarray:
+    """Gap between the k-th and (k+1)-th largest logit of each token."""
+    s = -np.sort(-np.asarray(logits, dtype=np.float64), axis=1)
+    return s[:, top_k - 1] - s[:, top_k]
+
+
+# ----------------------------------------------------------------------------
+# [Routing] capacity-factor dispatch
+# ----------------------------------------------------------------------------
+def capacity(T: int, top_k: int, E: int, capacity_factor: float) -> int:
+    """Per-expert capacity ceil(cf * T * k / E); +inf means every assignment fits."""
+    if math.isinf(capacity_factor):
+        return int(T)
+    return int(math.ceil(capacity_factor * float(T * top_k) / float(E)))
+
+
+def dispatch(idx: np.ndarray, w: np.ndarray, E: int, cap: int):
+    """Group assignments by expert with the capacity rule.
+
+    Tokens are visited in index order; assignment (t, j) to e = idx[t, j] is
+    kept iff fewer than ``cap`` assignments to e were kept before it.  Kept
+    assignments of expert e occupy consecutive slots offsets[e] + rank, in token
+    order (the grouping step of ``_dispatch_and_combine``, [Arch]).
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    kept = np.zeros(E, dtype=np.int64)
+    rank = np.full((T, k), -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if kept[e] < cap:
+                rank[t, j] = kept[e]
+                kept[e] += 1
+    counts_raw = np.bincount(idx.ravel().astype(np.int64), minlength=E)[:E]
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept)
+    n_kept = int(offsets[E])
+    slot_of = np.full((T, k), -1, dtype=np.int64)
+    perm = np.full(n_kept, -1, dtype=np.int64)
+    row_scale = np.zeros(n_kept, dtype=np.float64)
+    for t in range(T):
+        for j in range(k):
+            if rank[t, j] >= 0:
+                s = offsets[int(idx[t, j])] + rank[t, j]
+                slot_of[t, j] = s
+                perm[s] = t
+                row_scale[s] = w[t, j]
+    return {
+        "counts_raw": counts_raw.astype(np.int64),
+        "counts_kept": kept,
+        "offsets": offsets,
+        "perm": perm,
+        "slot_of": slot_of,
+        "row_scale": row_scale,
+        "n_kept": n_kept,
+        "dropped": int(T * k - n_kept),
+    }
+
+
+# ----------------------------------------------------------------------------
+# [Expert] SwiGLU expert
+# ----------------------------------------------------------------------------
+def silu(z: np.ndarray) -> np.ndarray:
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z))."""
+    return z / (1.0 + np.exp(-z))
+
+
+def swiglu_hidden(x_rows, w_gate_e, w_up_e) -> np.ndarray:
+    """H = silu(x @ W_gate) * (x @ W_up)   (SwiGLUExpert.forward, [Expert]).
+
+    Weights are stored [d, f] so that x @ W maps hidden -> expert_dim.
+    """
+    x = to_f64(x_rows)
+    return silu(x @ to_f64(w_gate_e)) * (x @ to_f64(w_up_e))
+
+
+def swiglu_expert(x_rows, w_gate_e, w_up_e, w_down_e) -> np.ndarray:
+    """y = (silu(x @ W_gate) * (x @ W_up)) @ W_down   ([Expert]); W_down is [f, d]."""
+    return swiglu_hidden(x_rows, w_gate_e, w_up_e) @ to_f64(w_down_e)
+
+
+# ----------------------------------------------------------------------------
+# [Arch] the whole layer
+# ----------------------------------------------------------------------------
+def layer_forward(x, w_router, w_gate, w_up, w_down, capacity_factor, logit_bias=None,
+                  top_k: int = 2, tokens=None, keep_hidden: bool = False):
+    """Forward pass of one MoE layer, returning every intermediate.
+
+    Router, top-k and dispatch run over all T tokens.  The expert FFN and the
+    combine run for the tokens in ``tokens`` (default: all), so large layers
+    can be checked on a subsample.  out[t] = sum over kept (t, j) of
+    w[t, j] * expert_{idx[t, j]}(x[t])  ([Arch] combine, [EP] weight scaling);
+    a token with no kept assignment outputs zero.
+    """
+    x = np.asarray(x)
+    T = x.shape[0]
+    E = np.asarray(w_router).shape[0]
+    lg = router_logits(x, w_router, logit_bias)
+    idx, w = top2_softmax(lg, top_k)
+    cap = capacity(T, top_k, E, capacity_factor)
+    disp = dispatch(idx, w, E, cap)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    d = x.shape[1]
+    out = np.zeros((tok.size, d), dtype=np.float64)
+    hidden = {}
+    for e in range(E):
+        rows = [(i, j) for i, t in enumerate(tok) for j in range(top_k)
+                if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
+        if not rows:
+            continue
+        xr = x[[tok[i] for i, _ in rows]]
+        h = swiglu_hidden(xr, w_gate[e], w_up[e])
+        y = h @ to_f64(w_down[e])
+        for r, (i, j) in enumerate(rows):
+            out[i] += w[tok[i], j] * y[r]
+            if keep_hidden:
+                hidden[int(disp["slot_of"][tok[i], j])] = h[r]
+    res = dict(disp)
+    res.update({"logits": lg, "idx": idx, "w": w, "cap": cap, "tokens": tok, "out": out})
+    if keep_hidden:
+        res["hidden"] = hidden
+    return res
+
+
+# ----------------------------------------------------------------------------
+# statistics the pages define
+# ----------------------------------------------------------------------------
+def expert_batch_size(global_batch: int, seq_len: int, num_experts: int = 8, top_k: int = 2) -> float:
+    """Average tokens per expert = batch * seq * k / E   ([Trade])."""
+    return global_batch * seq_len * top_k / num_experts
+
+
+def expert_utilization(counts, num_experts: int = 8, top_k: int = 2) -> np.ndarray:
+    """Assignments per expert normalised so that a balanced router gives 1.0 ([Dyn]).
+
+    utilization[e] = counts[e] / n_tokens * E / k with n_tokens = sum(counts) / k.
+    The page's snippet divides by the number of assignments (tokens * k) instead,
+    which would give 0.5 for a balanced router; its own comment says 1.0, and
+    that is the reading taken here.
+    """
+    c = np.asarray(counts, dtype=np.float64)
+    n_tokens = c.sum() / top_k
+    return c / n_tokens * num_experts / top_k

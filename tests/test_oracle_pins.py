@@ -1,0 +1,358 @@
+"""Pins of the CPU oracle against brute force, closed forms and the pages' values.
+
+Each check is written as a function of an oracle object so that the last test
+can plant plausible mistakes in a copy of the oracle and show that some pin
+fails for every one of them.
+"""
+import copy
+import itertools
+import json
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+
+import oracle.moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# brute-force helpers (pure Python loops, no numpy linear algebra)
+# ----------------------------------------------------------------------------
+def bf_logits(x, wr, bias=None):
+    T, d = len(x), len(x[0])
+    E = len(wr)
+    out = [[0.0] * E for _ in range(T)]
+    for t in range(T):
+        for e in range(E):
+            s = 0.0
+            for i in range(d):
+                s += float(x[t][i]) * float(wr[e][i])
+            out[t][e] = s + (0.0 if bias is None else float(bias[e]))
+    return out
+
+
+def bf_top2(row):
+    """The unique pair whose members both beat every other expert under (logit desc, index asc)."""
+    E = len(row)
+
+    def beats(a, b):
+        return row[a] > row[b] or (row[a] == row[b] and a < b)
+
+    found = []
+    for a, b in itertools.combinations(range(E), 2):
+        if all(beats(a, c) and beats(b, c) for c in range(E) if c not in (a, b)):
+            found.append((a, b) if beats(a, b) else (b, a))
+    assert len(found) == 1
+    return found[0]
+
+
+def bf_matvec(v, m):
+    """v [n] times m [n][p] -> [p]."""
+    p = len(m[0])
+    out = [0.0] * p
+    for i in range(len(v)):
+        vi = float(v[i])
+        row = m[i]
+        for j in range(p):
+            out[j] += vi * float(row[j])
+    return out
+
+
+def bf_expert(xt, wg, wu, wd):
+    g = bf_matvec(xt, wg)
+    u = bf_matvec(xt, wu)
+    h = [gi / (1.0 + math.exp(-gi)) * ui for gi, ui in zip(g, u)]
+    return bf_matvec(h, wd)
+
+
+def bf_layer(x, wr, wg, wu, wd, cap, bias=None):
+    """Every expert evaluated densely on every token, masked by brute-force top-2 and rank."""
+    lg = bf_logits(x, wr, bias)
+    T, d, E = len(x), len(x[0]), len(wr)
+    out = [[0.0] * d for _ in range(T)]
+    pairs = [bf_top2(r) for r in lg]
+    for t in range(T):
+        l0, l1 = lg[t][pairs[t][0]], lg[t][pairs[t][1]]
+        w = {pairs[t][0]: 1.0 / (1.0 + math.exp(l1 - l0)), pairs[t][1]: 1.0 / (1.0 + math.exp(l0 - l1))}
+        for e in range(E):
+            if e not in w:
+                continue
+            earlier = sum(1 for s in range(t) if e in pairs[s])  # rank among all earlier routings to e
+            if earlier >= cap:
+                continue
+            y = bf_expert(x[t], wg[e], wu[e], wd[e])
+            for i in range(d):
+                out[t][i] += w[e] * y[i]
+    return lg, pairs, out
+
+
+def rand_layer(rng, T, d, f, E, scale_r=1.0):
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) * scale_r
+    wg = rng.standard_normal((E, d, f)) / math.sqrt(d)
+    wu = rng.standard_normal((E, d, f)) / math.sqrt(d)
+    wd = rng.standard_normal((E, f, d)) / math.sqrt(f)
+    return x, wr, wg, wu, wd
+
+
+# ----------------------------------------------------------------------------
+# the pins, as functions of an oracle object
+# ----------------------------------------------------------------------------
+def pin_router_logits(o):
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 7))
+    wr = rng.standard_normal((8, 7))
+    bias = rng.standard_normal(8)
+    np.testing.assert_allclose(o.router_logits(x, wr), bf_logits(x, wr), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o.router_logits(x, wr, bias), bf_logits(x, wr, bias), rtol=0, atol=1e-12)
+
+
+def pin_top2_brute_force(o):
+    rng = np.random.default_rng(2)
+    # small integer logits make exact ties frequent
+    lg = rng.integers(-3, 4, size=(400, 8)).astype(np.float64)
+    idx, _ = o.top2_softmax(lg)
+    for t in range(lg.shape[0]):
+        assert tuple(idx[t]) == bf_top2(list(lg[t])), t
+
+
+def pin_softmax_closed_form(o):
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((300, 8)) * 2
+    idx, w = o.top2_softmax(lg)
+    l0 = lg[np.arange(300), idx[:, 0]]
+    l1 = lg[np.arange(300), idx[:, 1]]
+    np.testing.assert_allclose(w[:, 0], 1.0 / (1.0 + np.exp(l1 - l0)), rtol=1e-13, atol=0)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    assert np.all(w[:, 0] >= w[:, 1])
+
+
+def pin_zero_router(o):
+    x = np.random.default_rng(4).standard_normal((6, 16))
+    idx, w = o.top2_softmax(o.router_logits(x, np.zeros((8, 16))))
+    assert np.all(idx == np.array([0, 1])) and np.all(w == 0.5)
+
+
+def pin_scale_invariance(o):
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((50, 12))
+    wr = rng.standard_normal((8, 12))
+    a, _ = o.top2_softmax(o.router_logits(x, wr))
+    b, _ = o.top2_softmax(o.router_logits(x, 3.5 * wr))
+    np.testing.assert_array_equal(a, b)
+
+
+def pin_capacity_values(o):
+    assert o.capacity(64, 2, 8, 1.25) == 20
+    assert o.capacity(2048, 2, 8, 1.25) == 640
+    assert o.capacity(8192, 2, 8, 4.0) == 8192
+    assert o.capacity(16384, 2, 8, 1.25) == 5120
+    assert o.capacity(10, 2, 8, 1.0) == 3          # 2.5 rounds up
+    assert o.capacity(32, 2, 8, float("inf")) == 32
+
+
+def pin_dispatch_brute_force(o):
+    rng = np.random.default_rng(6)
+    for T, E, cap in [(40, 8, 7), (64, 8, 20), (33, 4, 5), (17, 8, 100)]:
+        idx = np.stack([rng.choice(E, 2, replace=False) for _ in range(T)]).astype(np.int32)
+        w = rng.random((T, 2))
+        r = o.dispatch(idx, w, E, cap)
+        slot_of, perm, off = r["slot_of"], r["perm"], r["offsets"]
+        kept_count = np.zeros(E, dtype=int)
+        for t in range(T):
+            for j in range(2):
+                e = idx[t, j]
+                earlier = sum(1 for s in range(t) if e in idx[s])
+                keep = earlier < cap
+                assert (slot_of[t, j] >= 0) == keep
+                if keep:
+                    assert slot_of[t, j] == off[e] + earlier
+                    assert perm[slot_of[t, j]] == t
+                    assert r["row_scale"][slot_of[t, j]] == w[t, j]
+                    kept_count[e] += 1
+        np.testing.assert_array_equal(r["counts_kept"], kept_count)
+        np.testing.assert_array_equal(r["counts_raw"], np.bincount(idx.ravel(), minlength=E))
+        assert np.all(r["counts_kept"] <= cap)
+        assert r["n_kept"] == int((slot_of >= 0).sum())
+        assert sorted(perm.tolist()) == sorted(int(t) for t, j in zip(*np.nonzero(slot_of >= 0)))
+        assert sorted(slot_of[slot_of >= 0].tolist()) == list(range(r["n_kept"]))
+
+
+def pin_no_drop(o):
+    rng = np.random.default_rng(7)
+    T = 64
+    idx = np.stack([rng.choice(8, 2, replace=False) for _ in range(T)]).astype(np.int32)
+    r = o.dispatch(idx, rng.random((T, 2)), 8, o.capacity(T, 2, 8, 8 / 2))
+    assert r["dropped"] == 0 and r["n_kept"] == 2 * T
+
+
+def pin_hand_built_drop(o):
+    # 8 tokens, every one routed to experts (0, 1); capacity 3 keeps tokens 0-2 only
+    T, d, f = 8, 4, 3
+    rng = np.random.default_rng(8)
+    x = np.abs(rng.standard_normal((T, d))) + 0.1
+    wr = np.zeros((8, d))
+    wr[0] = 2.0
+    wr[1] = 1.0
+    _, _, wg, wu, wd = rand_layer(rng, T, d, f, 8)
+    cf = 3 * 8 / (T * 2)  # ceil(cf*T*k/E) = 3
+    assert o.capacity(T, 2, 8, cf) == 3
+    r = o.layer_forward(x, wr, wg, wu, wd, cf)
+    assert np.all(r["idx"] == np.array([0, 1]))
+    assert list(r["slot_of"][:, 0]) == [0, 1, 2, -1, -1, -1, -1, -1]
+    assert list(r["slot_of"][:, 1]) == [3, 4, 5, -1, -1, -1, -1, -1]
+    assert np.all(r["out"][3:] == 0.0)
+    assert np.all(np.abs(r["out"][:3]).sum(axis=1) > 0)
+
+
+def pin_layer_dense_brute_force(o):
+    rng = np.random.default_rng(9)
+    T, d, f, E = 9, 5, 6, 8
+    x, wr, wg, wu, wd = rand_layer(rng, T, d, f, E)
+    bias = rng.standard_normal(E) * 0.3
+    for cf in (1.0, 2.0, float("inf")):
+        cap = o.capacity(T, 2, E, cf)
+        lg, pairs, out = bf_layer(x.tolist(), wr.tolist(), wg.tolist(), wu.tolist(), wd.tolist(), cap, bias)
+        r = o.layer_forward(x, wr, wg, wu, wd, cf, logit_bias=bias)
+        assert [tuple(p) for p in r["idx"]] == pairs
+        np.testing.assert_allclose(r["out"], out, rtol=1e-12, atol=1e-12)
+
+
+def pin_identity_experts(o):
+    # d = f and W_gate = W_up = W_down = I: each expert computes silu(x) * x
+    rng = np.random.default_rng(10)
+    T, d, E = 12, 6, 8
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d))
+    eye = np.broadcast_to(np.eye(d), (E, d, d)).copy()
+    r = o.layer_forward(x, wr, eye, eye, eye, float("inf"))
+    np.testing.assert_allclose(r["out"], x / (1 + np.exp(-x)) * x, rtol=1e-13, atol=1e-14)
+
+
+def pin_two_expert_dense(o):
+    # E = k = 2, cf = 1: every token goes to both experts, nothing is dropped
+    rng = np.random.default_rng(11)
+    T, d, f = 10, 4, 7
+    x, wr, wg, wu, wd = rand_layer(rng, T, d, f, 2)
+    r = o.layer_forward(x, wr, wg, wu, wd, 1.0)
+    lg = x @ wr.T
+    w0 = 1 / (1 + np.exp(lg[:, 1] - lg[:, 0]))
+    y = []
+    for e in range(2):
+        ye = np.array([bf_expert(x[t], wg[e].tolist(), wu[e].tolist(), wd[e].tolist()) for t in range(T)])
+        y.append(ye)
+    np.testing.assert_allclose(r["out"], w0[:, None] * y[0] + (1 - w0)[:, None] * y[1], rtol=1e-12, atol=1e-12)
+
+
+def pin_bf16_decoding(o):
+    bits = np.array([0x3F80, 0xC000, 0x3E80, 0x0000, 0x8000, 0x4049], dtype=np.uint16)
+    np.testing.assert_array_equal(o.to_f64(bits), [1.0, -2.0, 0.25, 0.0, -0.0, 3.140625])
+
+
+ALL_PINS = [pin_router_logits, pin_top2_brute_force, pin_softmax_closed_form, pin_zero_router,
+            pin_scale_invariance, pin_capacity_values, pin_dispatch_brute_force, pin_no_drop,
+            pin_hand_built_drop, pin_layer_dense_brute_force, pin_identity_experts,
+            pin_two_expert_dense, pin_bf16_decoding]
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(pin):
+    pin(O)
+
+
+def test_expert_batch_size_golden():
+    with open(os.path.join(GOLDEN, "expert_batch_size.json")) as fh:
+        g = json.load(fh)
+    for c in g["cases"]:
+        assert O.expert_batch_size(c["global_batch"], c["seq_len"]) == c["tokens_per_expert"]
+
+
+def test_utilization_balanced_is_one():
+    np.testing.assert_allclose(O.expert_utilization([250] * 8), 1.0)
+    u = O.expert_utilization([400, 100, 250, 250, 250, 250, 250, 250])
+    assert u[0] == pytest.approx(1.6) and u.sum() == pytest.approx(8 / 2 * 2)
+
+
+def test_near_tie_gap():
+    lg = np.array([[3.0, 1.0, 2.0, 0.5, 0, 0, 0, 0]])
+    assert O.near_tie_gap(lg)[0] == pytest.approx(1.0)
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: each mutant of the oracle must fail at least one pin
+# ----------------------------------------------------------------------------
+def _mutant(**overrides):
+    m = types.SimpleNamespace(**{k: getattr(O, k) for k in dir(O) if not k.startswith("_")})
+    for k, v in overrides.items():
+        setattr(m, k, v)
+    # layer_forward must call the mutated pieces
+    def layer_forward(x, w_router, w_gate, w_up, w_down, capacity_factor, logit_bias=None,
+                      top_k=2, tokens=None, keep_hidden=False):
+        saved = {k: getattr(O, k) for k in overrides}
+        try:
+            for k, v in overrides.items():
+                setattr(O, k, v)
+            return saved.get("layer_forward", O.layer_forward)(
+                x, w_router, w_gate, w_up, w_down, capacity_factor, logit_bias, top_k, tokens, keep_hidden)
+        finally:
+            for k, v in saved.items():
+                setattr(O, k, v)
+    m.layer_forward = layer_forward
+    return m
+
+
+def _top2_ascending_ties(lg, top_k=2):
+    lg = np.asarray(lg, dtype=np.float64)
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :top_k]
+    # ties resolved toward the higher index
+    rev = lg.shape[1] - 1 - np.argsort(-lg[:, ::-1], axis=1, kind="stable")[:, :top_k]
+    sel = np.take_along_axis(lg, rev, axis=1)
+    ex = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return rev.astype(np.int32), ex / ex.sum(axis=1, keepdims=True)
+
+
+def _softmax_all8(lg, top_k=2):
+    lg = np.asarray(lg, dtype=np.float64)
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :top_k]
+    p = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p = p / p.sum(axis=1, keepdims=True)
+    return order.astype(np.int32), np.take_along_axis(p, order, axis=1)
+
+
+def _dispatch_off_by_one(idx, w, E, cap):
+    return _orig_dispatch(idx, w, E, cap + 1)
+
+
+_orig_dispatch = O.dispatch
+_orig_silu = O.silu
+_orig_router = O.router_logits
+_orig_hidden = O.swiglu_hidden
+_orig_capacity = O.capacity
+
+MUTANTS = {
+    "silu_is_identity": dict(silu=lambda z: z),
+    "sigmoid_sign_flipped": dict(silu=lambda z: z / (1.0 + np.exp(z))),
+    "router_bias_dropped": dict(router_logits=lambda x, wr, b=None: _orig_router(x, wr, None)),
+    "router_transposed_scale": dict(router_logits=lambda x, wr, b=None: 2 * _orig_router(x, wr, b)),
+    "ties_to_higher_index": dict(top2_softmax=_top2_ascending_ties),
+    "softmax_over_all_experts": dict(top2_softmax=_softmax_all8),
+    "capacity_off_by_one": dict(dispatch=_dispatch_off_by_one),
+    "capacity_floor": dict(capacity=lambda T, k, E, cf: T if math.isinf(cf) else int(math.floor(cf * T * k / E))),
+    "gate_up_swapped": dict(swiglu_hidden=lambda x, g, u: _orig_hidden(x, u, g)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    m = _mutant(**MUTANTS[name])
+    failures = 0
+    for pin in ALL_PINS:
+        try:
+            pin(m)
+        except AssertionError:
+            failures += 1
+    assert failures >= 1, f"no pin catches mutant {name}"
