@@ -1,0 +1,408 @@
+"""Benchmark of the MoE layer forward pass on B200.
+
+One step = one pass of the whole layer (router + top-2, dispatch, gather,
+gate/up + SwiGLU, down, combine) over one batch of the workload, through the
+C ABI.  Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Workload default: the Grok-1-shape prefill layer (T=8192, d=6144, f=32768,
+E=8, top-2, no drop).  Under torchrun every rank runs its own batch (distinct
+x, same weights): the layer shards by token batch with no collective on the
+data path ("weak" scaling); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import configs  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks/throttle reasons for one GPU while running."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 8 and (not self.uuid or parts[0] == self.uuid):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i] == "Active"})
+        pw = [float(r[3]) for r in self.rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------- CPU baseline (oracle)
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(w, host, x, n_tokens, seed):
+    """Time the oracle on a seeded token sample of this workload (routing over all T)."""
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    tok = np.sort(rng.choice(w.T, size=min(n_tokens, w.T), replace=False))
+    t0 = time.perf_counter()
+    oracle.layer_forward(x, host["wr"], host["wg"], host["wu"], host["wd"], w.capacity_factor,
+                         logit_bias=configs.make_bias(w), tokens=tok)
+    return time.perf_counter() - t0, len(tok)
+
+
+def reference_arm(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    host = dict(wr=configs.make_router(w), wg=configs.make_w_gate(w), wu=configs.make_w_up(w),
+                wd=configs.make_w_down(w))
+    x = configs.make_x(w)
+    per_step = args.ref_tokens
+    for i in range(args.warmup):
+        oracle_sample(w, host, x, per_step, 1000 + i)
+    tot, ntok = 0.0, 0
+    for i in range(args.steps):
+        t, n = oracle_sample(w, host, x, per_step, i)
+        tot += t
+        ntok += n
+    value = ntok / tot
+    cores = blas_threads()
+    sample = (f"oracle (fp64 numpy) per step: router, top-2 and dispatch over all T={w.T} tokens, "
+              f"expert FFN and combine for {per_step} seeded tokens")
+    line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "T": w.T, "d": w.d, "f": w.f, "E": w.E, "top_k": w.top_k,
+            "capacity_factor": w.capacity_factor, "logit_bias": list(w.logit_bias) if w.logit_bias else None,
+            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (3 * w.E * w.d * w.f * 2 / 1e9),
+            "description": w.description}
+
+
+# ---------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="grok_prefill", choices=sorted(configs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per reference-arm step")
+    ap.add_argument("--cpu-tokens", type=int, default=64, help="tokens in the CPU-baseline sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    w = configs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_moe_layer_07_b200 as moe
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+    # ---- inputs: weights generated once (rank 0) and broadcast; x distinct per rank
+    host = None
+    if rank == 0:
+        host = dict(wr=configs.make_router(w), wg=configs.make_w_gate(w), wu=configs.make_w_up(w),
+                    wd=configs.make_w_down(w))
+        W = {k: to_dev(v) for k, v in host.items()}
+    else:
+        tdt = torch.bfloat16 if w.storage == "bf16" else torch.float32
+        W = {"wr": torch.empty((w.E, w.d), dtype=tdt, device=dev),
+             "wg": torch.empty((w.E, w.d, w.f), dtype=tdt, device=dev),
+             "wu": torch.empty((w.E, w.d, w.f), dtype=tdt, device=dev),
+             "wd": torch.empty((w.E, w.f, w.d), dtype=tdt, device=dev)}
+    if world > 1:
+        for k in ("wr", "wg", "wu", "wd"):
+            dist.broadcast(W[k], src=0)
+    from synth import normal
+
+    x_np = configs.make_x(w) if rank == 0 else normal(configs.SEED, configs.TID_X + 1000 * rank, (w.T, w.d),
+                                                       dtype=w.storage)
+    x = to_dev(x_np)
+    bias = configs.make_bias(w)
+    bias_d = None if bias is None else to_dev(bias)
+    cfg = moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype=w.storage)
+    rows = w.T * w.top_k
+    tdt = cfg.torch_dtype
+    buf = {
+        "idx": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
+        "w": torch.empty((w.T, 2), dtype=torch.float32, device=dev),
+        "h": torch.empty((rows, w.f), dtype=tdt, device=dev),
+        "y": torch.empty((rows, w.d), dtype=torch.float32, device=dev),
+        "out": torch.empty((w.T, w.d), dtype=tdt, device=dev),
+        "ws": torch.empty((max(moe.dispatch_workspace_size(cfg), 16),), dtype=torch.uint8, device=dev),
+    }
+    disp = {"counts_raw": torch.empty(8, dtype=torch.int32, device=dev),
+            "counts_kept": torch.empty(8, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(9, dtype=torch.int32, device=dev),
+            "perm": torch.empty(rows, dtype=torch.int32, device=dev),
+            "slot_of": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
+            "row_scale": torch.empty(rows, dtype=torch.float32, device=dev),
+            "x_perm": torch.empty((rows, w.d), dtype=tdt, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+    names = ["router", "dispatch", "gate_up", "down", "combine"]
+    launches_per_step = 8  # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        moe.router_topk(cfg, x, W["wr"], bias_d, topk_idx=buf["idx"], topk_w=buf["w"])
+        if ev:
+            ev[1].record(stream)
+        moe.dispatch(cfg, x, buf["idx"], buf["w"], out=disp, ws=buf["ws"])
+        if ev:
+            ev[2].record(stream)
+        moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
+        if ev:
+            ev[3].record(stream)
+        moe.expert_down(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], y=buf["y"])
+        if ev:
+            ev[4].record(stream)
+        moe.combine(cfg, buf["y"], disp["slot_of"], buf["w"], weights_applied=True, out=buf["out"])
+        if ev:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    n_kept = int(disp["offsets"][-1].item())
+    counts_kept = disp["counts_kept"].cpu().tolist()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    uuid = ""
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.5)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    per_kernel = {n: 0.0 for n in names}
+    for e in evs:
+        for j, n in enumerate(names):
+            per_kernel[n] += e[j].elapsed_time(e[j + 1])
+    per_kernel = {n: v / args.steps for n, v in per_kernel.items()}
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens = world * w.T * args.steps
+    value = tokens / (ms_total / 1000.0)
+    flops_step = 2.0 * w.T * w.d * w.E + 6.0 * n_kept * w.d * w.f
+    tflops = world * flops_step * args.steps / (ms_total / 1000.0) / 1e12
+
+    peaks, peak_src = load_peaks()
+    gu_flops = 4.0 * n_kept * w.d * w.f
+    gu_ms = per_kernel["gate_up"]
+    achieved = gu_flops / (gu_ms / 1000.0) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "kernel": "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "traffic": None,
+                "algorithmic": f"4*d*f*N_kept = {gu_flops:.4e} FLOP per launch (N_kept={n_kept})",
+                "down": {"achieved": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12,
+                         "frac": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12 / peak}}
+
+    line = {"metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.storage == "bf16" else "f32",
+            "data": "synthetic (seeded Philox4x32-10 normal inputs, random-init weights)",
+            "config": workload_config(w), "tflops": tflops,
+            "tensor_frac_layer": tflops / peak,
+            "kernels_ms": per_kernel, "counts_kept": counts_kept, "n_kept": n_kept,
+            "gpu_launches": launches_per_step * args.steps, "roofline": roofline, "clocks": clk}
+
+    # ---- end to end: host x in, host out, through the C entry point with host buffers
+    if not args.no_e2e:
+        ws_full = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+        x_host = torch.from_numpy(np.ascontiguousarray(x_np))
+        x_host = (x_host.view(torch.bfloat16) if w.storage == "bf16" else x_host).pin_memory()
+        out_host = torch.empty((w.T, w.d), dtype=tdt).pin_memory()
+        for _ in range(2):
+            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_host, ws_full,
+                                   logit_bias=bias_d)
+        if world > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_host, ws_full,
+                                   logit_bias=bias_d)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        nbytes = w.T * w.d * (2 if w.storage == "bf16" else 4)
+        line["e2e"] = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                       "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms / args.steps,
+                       "api": "moe_layer_forward_host (pinned host x/out, device-resident weights)"}
+        del ws_full
+
+    # ---- decode (weight streaming) on the same Grok-shape weights
+    if not args.no_decode and w.name == "grok_prefill":
+        line["decode"] = decode_bench(moe, W, dev, stream, peaks, peak_src, world)
+
+    if rank == 0 and world == 1 and not args.no_cpu and host is not None:
+        t, n = oracle_sample(w, host, x_np, args.cpu_tokens, 7)
+        line["cpu_baseline"] = {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"oracle (fp64 numpy): router, top-2 and dispatch over all T={w.T} "
+                                          f"tokens, expert FFN and combine for {n} seeded tokens; "
+                                          f"value = {n} tokens / {t:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
+    import torch
+
+    w = configs.WORKLOADS["grok_decode"]
+    cfg = moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16")
+    xs = torch.stack([torch.from_numpy(configs.make_x(w, call=i)).view(torch.bfloat16) for i in range(w.calls)])
+    xs = xs.to(dev)
+    ws = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
+    stats = torch.zeros(26, dtype=torch.int32, device=dev)
+    used = torch.zeros(8, dtype=torch.int64, device=dev)
+    for i in range(3):
+        moe.layer_forward(cfg, xs[i], W["wr"], W["wg"], W["wu"], W["wd"], out=out, ws=ws)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(w.calls):
+        moe.layer_forward(cfg, xs[i], W["wr"], W["wg"], W["wu"], W["wd"], out=out, stats=stats, ws=ws)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    # experts used per call (counted after timing, on a second pass)
+    n_used = 0
+    for i in range(w.calls):
+        moe.layer_forward(cfg, xs[i], W["wr"], W["wg"], W["wu"], W["wd"], out=out, stats=stats, ws=ws)
+        used += (stats[8:16] > 0).to(torch.int64)
+    torch.cuda.synchronize(dev)
+    n_used = int(used.sum().item())
+    weight_bytes = n_used * 3 * w.d * w.f * 2
+    gbs = weight_bytes / (ms / 1000.0) / 1e9
+    return {"workload": w.name, "calls": w.calls, "ms_per_call": ms / w.calls,
+            "tokens_per_s": w.T * w.calls / (ms / 1000.0), "expert_weight_gb_per_call": weight_bytes / w.calls / 1e9,
+            "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm"}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * moe.h -- C ABI of a B200 (sm_100a) implementation of the forward pass of a
+ * Grok-1-style sparse mixture-of-experts SwiGLU FFN layer.
+ *
+ * The operation follows the page "How does Grok-1 use a mixture-of-experts
+ * design?" (n4n.ai):
+ *   - section "The high-level architecture", GrokMoELayer.forward: router
+ *     logits over 8 experts, top-2, softmax over the two selected logits,
+ *     dispatch to the experts and weighted combine back to token order;
+ *   - section "Routing: top-2 without auxiliary loss", grok_router_forward and
+ *     the paragraph after it: router weight stored [E, hidden], capacity factor
+ *     (1.25 in training; no dropping at inference);
+ *   - section "Expert implementation: SwiGLU at scale", SwiGLUExpert and
+ *     FusedSwiGLUExpert: y = W_down(silu(W_gate x) * W_up x), no bias.
+ * and the page "Let Grok spill the beans on Grok", whose feature list states
+ * that the layer output is the weighted sum of the active experts' outputs.
+ *
+ * Readings where the pages leave a step open:
+ *   capacity = ceil(capacity_factor * T * top_k / E), computed in double in that
+ *   order (+INFINITY: no drop); overflow is dropped lowest token index first;
+ *   routing weights are not renormalised after a drop; a token with both
+ *   assignments dropped outputs zero; equal logits rank the lower expert first.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; every other buffer pointer is
+ *     device memory owned by the caller.  The library never allocates, frees
+ *     or keeps a pointer after a call returns.
+ *   - Tensors are dense row-major.  Buffers must be 16-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t); calls return before the
+ *     GPU finishes, except moe_layer_forward_host and moe_get_device_error.
+ *   - Argument errors are reported synchronously, before anything is launched:
+ *     MOE_ERR_INVALID_ARG (null pointer, bad size, misalignment),
+ *     MOE_ERR_UNSUPPORTED (E != 8, top_k != 2, d or f not a multiple of 128
+ *     for bf16 / 64 for fp32), MOE_ERR_WORKSPACE (workspace too small).
+ *     A failed launch returns MOE_ERR_CUDA.  Inputs are never modified.
+ *   - Checks made by the kernels themselves (an expert index outside [0, E),
+ *     a slot outside the buffers, inconsistent offsets, a pipeline wait that
+ *     timed out) do not trap: the offending element is skipped and a device
+ *     error word is set, read back with moe_get_device_error().
+ *   - T == 0 is valid and launches nothing.
+ */
+#ifndef SPARSE_MOE_LAYER_07_B200_MOE_H
+#define SPARSE_MOE_LAYER_07_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_DEVICE_CHECK = 5,
+  MOE_ERR_TIMEOUT = 6
+} moe_status_t;
+
+/* Storage and arithmetic type of x, the weights and out.
+ * MOE_F32:  fp32 everywhere (hidden activation H in fp32).
+ * MOE_BF16: bf16 storage, fp32 accumulation, H rounded once to bf16. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Bits of the device error word. */
+#define MOE_DEVERR_EXPERT_INDEX 0x1 /* an expert id outside [0, E) */
+#define MOE_DEVERR_SLOT_INDEX 0x2   /* a slot outside [0, T*top_k) */
+#define MOE_DEVERR_OFFSETS 0x4      /* expert offsets not monotone or too large */
+#define MOE_DEVERR_TIMEOUT 0x8      /* a pipeline wait ran past its limit */
+
+/* Layer hyper-parameters ("GrokMoELayer" in the architecture section:
+ * num_experts 8, top_k 2, hidden_size, expert_dim). */
+typedef struct {
+  int64_t T;              /* tokens = batch * seq_len */
+  int64_t d;              /* hidden_size */
+  int64_t f;              /* expert_dim */
+  int32_t E;              /* num_experts; must be 8 */
+  int32_t top_k;          /* must be 2 */
+  double capacity_factor; /* > 0; +INFINITY means no drop */
+  int32_t dtype;          /* moe_dtype_t */
+  int32_t reserved;       /* must be 0 */
+} moe_config_t;
+
+/* Length of the stats array written by moe_layer_forward (int32):
+ * [0, E) counts_raw, [E, 2E) counts_kept, [2E, 3E+1) offsets, [3E+1] dropped. */
+#define MOE_STATS_LEN(E) (3 * (E) + 2)
+
+/* Version of this ABI (incremented on incompatible change). */
+MOE_API int32_t moe_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Per-expert capacity min(T, ceil(capacity_factor * T * top_k / E)) (T when the
+ * factor is +INFINITY; no expert can receive more than T assignments), as used
+ * by moe_dispatch; -1 for an invalid config.
+ * Definition: capacity paragraph of "Routing: top-2 without auxiliary loss". */
+MOE_API int64_t moe_capacity(const moe_config_t* cfg);
+
+/* Bytes of device workspace needed by moe_dispatch (per-block histograms). */
+MOE_API size_t moe_dispatch_workspace_size(const moe_config_t* cfg);
+
+/* Bytes of device workspace needed by moe_expert_ffn / moe_expert_down. */
+MOE_API size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg);
+
+/* Bytes of device workspace needed by moe_layer_forward and
+ * moe_layer_forward_host (all intermediates); 0 for an invalid config. */
+MOE_API size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Router and top-2 ("Routing: top-2 without auxiliary loss",
+ * grok_router_forward; "The high-level architecture", forward):
+ *   logits[t, e] = sum_i x[t, i] * w_router[e, i]  (+ logit_bias[e])
+ *   topk_idx[t, 0..1] = the two largest logits, descending, ties to lower e
+ *   topk_w[t, j]      = softmax over the two selected logits
+ * x [T, d] and w_router [E, d] in cfg->dtype; accumulation in fp32.
+ * logit_bias [E] fp32 or NULL; logits [T, E] fp32 or NULL (not written);
+ * topk_idx [T, 2] int32; topk_w [T, 2] fp32. */
+MOE_API moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router,
+                             const float* logit_bias, float* logits, int32_t* topk_idx,
+                             float* topk_w, moe_stream_t stream);
+
+/* Capacity-factor dispatch (the "_apply_capacity" and grouping steps of
+ * grok_router_forward / _dispatch_and_combine):
+ *   counts_raw[e]  = number of assignments routed to e
+ *   rank(t, e)     = number of tokens t' < t routed to e
+ *   kept iff rank < capacity;   counts_kept[e] = min(counts_raw[e], capacity)
+ *   offsets        = exclusive prefix sum of counts_kept (E + 1 entries)
+ *   slot_of[t, j]  = offsets[e] + rank for a kept assignment, else -1
+ *   perm[slot] = t,  row_scale[slot] = topk_w[t, j]
+ *   x_perm[slot, :] = x[perm[slot], :]   (skipped when x_perm is NULL)
+ * perm, row_scale: [T*2] (the first offsets[E] entries are written);
+ * slot_of [T, 2]; x_perm [T*2, d] in cfg->dtype.  ws: moe_dispatch_workspace_size
+ * bytes of scratch.  Deterministic: no atomics decide any output. */
+MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                          const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
+                          int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
+                          void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* SwiGLU expert FFN over the grouped rows ("Expert implementation: SwiGLU at
+ * scale", SwiGLUExpert / FusedSwiGLUExpert), for each expert e and each row r
+ * in [offsets[e], offsets[e+1]):
+ *   h[r, :] = silu(x_perm[r, :] @ w_gate[e]) * (x_perm[r, :] @ w_up[e])
+ *   y[r, :] = row_scale[r] * (h[r, :] @ w_down[e])      (row_scale NULL: 1)
+ * w_gate, w_up [E, d, f]; w_down [E, f, d]; x_perm [T*2, d]; h [T*2, f], all in
+ * cfg->dtype; y [T*2, d] fp32.  offsets is the device array from moe_dispatch.
+ * bf16 runs on the tensor cores with fp32 accumulation; h is rounded once. */
+MOE_API moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                            const void* w_gate, const void* w_up, const void* w_down,
+                            const float* row_scale, void* h, float* y, void* ws, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* The two halves of moe_expert_ffn, for callers that time or overlap them:
+ * gate/up with the fused SwiGLU epilogue (writes h), and down (writes y). */
+MOE_API moe_status_t moe_expert_gate_up(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                                const void* w_gate, const void* w_up, void* h, moe_stream_t stream);
+MOE_API moe_status_t moe_expert_down(const moe_config_t* cfg, const void* h, const int32_t* offsets,
+                             const void* w_down, const float* row_scale, float* y, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* Weighted combine back to token order ("The high-level architecture",
+ * _dispatch_and_combine; weighted sum of the active experts' outputs):
+ *   out[t, :] = sum over j = 0, 1 with slot_of[t, j] >= 0 of
+ *               s_j * y[slot_of[t, j], :]      (fp32, j = 0 first)
+ * with s_j = 1 when weights_applied != 0 (y already carries the routing
+ * weight) and s_j = topk_w[t, j] otherwise.  out [T, d] in cfg->dtype
+ * (rounded once); a token with no kept assignment gets zeros. */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const float* y, const int32_t* slot_of,
+                         const float* topk_w, int32_t weights_applied, void* out,
+                         moe_stream_t stream);
+
+/* The whole layer forward: router -> dispatch -> expert FFN -> combine.
+ * x [T, d]; w_router [E, d]; w_gate/w_up [E, d, f]; w_down [E, f, d]; out [T, d];
+ * logit_bias [E] fp32 or NULL; stats: device int32[MOE_STATS_LEN(E)] or NULL.
+ * ws: moe_workspace_size(cfg) bytes of device scratch, owned by the caller. */
+MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router,
+                               const float* logit_bias, const void* w_gate, const void* w_up,
+                               const void* w_down, void* out, int32_t* stats, void* ws,
+                               size_t ws_bytes, moe_stream_t stream);
+
+/* moe_layer_forward with x and out in host memory: copies x_host to the device
+ * (inside ws), runs the layer, copies the result to out_host and waits for the
+ * stream.  Weights, logit_bias and ws are device memory.  Page-locked host
+ * buffers make the copies asynchronous with respect to other work. */
+MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host, const void* w_router,
+                                    const float* logit_bias, const void* w_gate, const void* w_up,
+                                    const void* w_down, void* out_host, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* Waits for the current device, returns the device error word (MOE_DEVERR_*
+ * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.
+ * Returns MOE_ERR_DEVICE_CHECK when the word is non-zero, else MOE_OK. */
+MOE_API moe_status_t moe_get_device_error(int32_t* code, int32_t clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_MOE_LAYER_07_B200_MOE_H */

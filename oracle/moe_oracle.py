@@ -38,6 +38,7 @@ Parity unpinned: none (each function is pinned by tests/test_oracle_pins.py).
 from __future__ import annotations
 
 import math
+import sys
 
 import numpy as np
 
@@ -46,11 +47,19 @@ import numpy as np
 # input decoding (storage format only)
 # ----------------------------------------------------------------------------
 def to_f64(a: np.ndarray) -> np.ndarray:
-    """Widen stored inputs to float64: uint16 arrays hold bf16 bit patterns."""
+    """Widen stored inputs to float64 (exact): uint16 arrays hold bf16 bit patterns.
+
+    A bf16 value is the high half of the fp32 with the same bits, so the bf16
+    bits are written into the high 16 bits of zeroed 32-bit words (little-endian
+    layout) and the result is read as fp32 and widened to fp64.
+    """
     a = np.asarray(a)
     if a.dtype == np.uint16:
-        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    return a.astype(np.float64)
+        assert sys.byteorder == "little"
+        w = np.zeros(a.shape, dtype=np.uint32)
+        w.view(np.uint16)[..., 1::2] = a
+        return w.view(np.float32).astype(np.float64)
+    return np.asarray(a, dtype=np.float64)
 
 
 # ----------------------------------------------------------------------------

@@ -1,0 +1,264 @@
+"""B200-native forward pass of a Grok-1-style top-2 sparse MoE SwiGLU layer.
+
+Thin ctypes binding over ``libmoe_b200.so`` (C ABI declared in
+``include/moe.h``).  The functions below carry the same names as the C entry
+points without the ``moe_`` prefix; they only check and marshal arguments
+(tensor pointers, the current CUDA stream) and allocate output tensors with
+PyTorch when the caller does not pass them.  Every step of the layer runs in
+the library's CUDA kernels: there is no fallback of any kind, and importing
+this package fails if the library has not been built
+(``python -m sparse_moe_layer_07_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "MoEError", "Config", "LIB_PATH", "lib", "abi_version", "capacity", "workspace_size",
+    "dispatch_workspace_size", "router_topk", "dispatch", "expert_ffn", "expert_gate_up",
+    "expert_down", "combine", "layer_forward", "layer_forward_host", "get_device_error",
+    "STATUS", "DEVERR",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
+DEVERR = {"EXPERT_INDEX": 0x1, "SLOT_INDEX": 0x2, "OFFSETS": 0x4, "TIMEOUT": 0x8}
+_DTYPES = {"f32": 0, "bf16": 1}
+_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class _CConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("f", ctypes.c_int64),
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_moe_layer_07_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    cfgp = ctypes.POINTER(_CConfig)
+    sz = ctypes.c_size_t
+    sig = {
+        "moe_abi_version": ([], ctypes.c_int32),
+        "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "moe_capacity": ([cfgp], ctypes.c_int64),
+        "moe_dispatch_workspace_size": ([cfgp], sz),
+        "moe_expert_ffn_workspace_size": ([cfgp], sz),
+        "moe_workspace_size": ([cfgp], sz),
+        "moe_router_topk": ([cfgp, P, P, P, P, P, P, P], ctypes.c_int),
+        "moe_dispatch": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_expert_ffn": ([cfgp, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_expert_gate_up": ([cfgp, P, P, P, P, P, P], ctypes.c_int),
+        "moe_expert_down": ([cfgp, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_combine": ([cfgp, P, P, P, ctypes.c_int32, P, P], ctypes.c_int),
+        "moe_layer_forward": ([cfgp, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_layer_forward_host": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+lib = _load()
+
+
+class Config:
+    """Layer hyper-parameters (``moe_config_t``)."""
+
+    def __init__(self, T: int, d: int, f: int, E: int = 8, top_k: int = 2,
+                 capacity_factor: float = 1.25, dtype: str = "bf16"):
+        if dtype not in _DTYPES:
+            raise ValueError(f"dtype must be one of {sorted(_DTYPES)}")
+        self.T, self.d, self.f, self.E, self.top_k = int(T), int(d), int(f), int(E), int(top_k)
+        self.capacity_factor = float(capacity_factor)
+        self.dtype = dtype
+        self._c = _CConfig(self.T, self.d, self.f, self.E, self.top_k, self.capacity_factor,
+                           _DTYPES[dtype], 0)
+
+    @property
+    def torch_dtype(self):
+        return _TORCH_DTYPE[self.dtype]
+
+    @property
+    def ref(self):
+        return ctypes.byref(self._c)
+
+    def __repr__(self):
+        return (f"Config(T={self.T}, d={self.d}, f={self.f}, E={self.E}, top_k={self.top_k}, "
+                f"capacity_factor={self.capacity_factor}, dtype={self.dtype!r})")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dev_ptr(t):
+    if t is not None and not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    return _ptr(t)
+
+
+def _stream(stream, device=None):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MoEError(status, where)
+
+
+def _empty(shape, dtype, like):
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+def abi_version() -> int:
+    return lib.moe_abi_version()
+
+
+def capacity(cfg: Config) -> int:
+    return lib.moe_capacity(cfg.ref)
+
+
+def workspace_size(cfg: Config) -> int:
+    return lib.moe_workspace_size(cfg.ref)
+
+
+def dispatch_workspace_size(cfg: Config) -> int:
+    return lib.moe_dispatch_workspace_size(cfg.ref)
+
+
+def router_topk(cfg: Config, x, w_router, logit_bias=None, logits=None, topk_idx=None, topk_w=None,
+                want_logits: bool = False, stream=None):
+    """Router logits, top-2 experts and their softmax weights.  Returns (idx, w, logits|None)."""
+    if topk_idx is None:
+        topk_idx = _empty((cfg.T, cfg.top_k), torch.int32, x)
+    if topk_w is None:
+        topk_w = _empty((cfg.T, cfg.top_k), torch.float32, x)
+    if logits is None and want_logits:
+        logits = _empty((cfg.T, cfg.E), torch.float32, x)
+    _check(lib.moe_router_topk(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(logit_bias), _dev_ptr(logits),
+                               _dev_ptr(topk_idx), _dev_ptr(topk_w), _stream(stream, x.device)), "moe_router_topk")
+    return topk_idx, topk_w, logits
+
+
+def dispatch(cfg: Config, x, topk_idx, topk_w, gather: bool = True, out=None, ws=None, stream=None):
+    """Capacity dispatch.  Returns a dict of counts_raw, counts_kept, offsets, perm, slot_of,
+    row_scale and x_perm (None when gather is False)."""
+    dev = topk_idx
+    rows = cfg.T * cfg.top_k
+    o = dict(out or {})
+    o.setdefault("counts_raw", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("counts_kept", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("offsets", _empty((cfg.E + 1,), torch.int32, dev))
+    o.setdefault("perm", _empty((rows,), torch.int32, dev))
+    o.setdefault("slot_of", _empty((cfg.T, cfg.top_k), torch.int32, dev))
+    o.setdefault("row_scale", _empty((rows,), torch.float32, dev))
+    if gather:
+        o.setdefault("x_perm", _empty((rows, cfg.d), cfg.torch_dtype, dev))
+    else:
+        o["x_perm"] = None
+    nbytes = dispatch_workspace_size(cfg)
+    if ws is None:
+        ws = _empty((max(nbytes, 1),), torch.uint8, dev)
+    _check(lib.moe_dispatch(cfg.ref, _dev_ptr(x), _dev_ptr(topk_idx), _dev_ptr(topk_w), _dev_ptr(o["counts_raw"]),
+                            _dev_ptr(o["counts_kept"]), _dev_ptr(o["offsets"]), _dev_ptr(o["perm"]),
+                            _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]), _dev_ptr(o["x_perm"]),
+                            _dev_ptr(ws), ws.numel(), _stream(stream, dev.device)), "moe_dispatch")
+    return o
+
+
+def expert_gate_up(cfg: Config, x_perm, offsets, w_gate, w_up, h=None, stream=None):
+    if h is None:
+        h = _empty((cfg.T * cfg.top_k, cfg.f), cfg.torch_dtype, x_perm)
+    _check(lib.moe_expert_gate_up(cfg.ref, _dev_ptr(x_perm), _dev_ptr(offsets), _dev_ptr(w_gate), _dev_ptr(w_up),
+                                  _dev_ptr(h), _stream(stream, x_perm.device)), "moe_expert_gate_up")
+    return h
+
+
+def expert_down(cfg: Config, h, offsets, w_down, row_scale=None, y=None, ws=None, stream=None):
+    if y is None:
+        y = _empty((cfg.T * cfg.top_k, cfg.d), torch.float32, h)
+    _check(lib.moe_expert_down(cfg.ref, _dev_ptr(h), _dev_ptr(offsets), _dev_ptr(w_down), _dev_ptr(row_scale),
+                               _dev_ptr(y), _dev_ptr(ws), 0 if ws is None else ws.numel(),
+                               _stream(stream, h.device)), "moe_expert_down")
+    return y
+
+
+def expert_ffn(cfg: Config, x_perm, offsets, w_gate, w_up, w_down, row_scale=None, h=None, y=None, ws=None,
+               stream=None):
+    """SwiGLU experts over the grouped rows.  Returns (h, y)."""
+    if h is None:
+        h = _empty((cfg.T * cfg.top_k, cfg.f), cfg.torch_dtype, x_perm)
+    if y is None:
+        y = _empty((cfg.T * cfg.top_k, cfg.d), torch.float32, x_perm)
+    _check(lib.moe_expert_ffn(cfg.ref, _dev_ptr(x_perm), _dev_ptr(offsets), _dev_ptr(w_gate), _dev_ptr(w_up),
+                              _dev_ptr(w_down), _dev_ptr(row_scale), _dev_ptr(h), _dev_ptr(y), _dev_ptr(ws),
+                              0 if ws is None else ws.numel(), _stream(stream, x_perm.device)), "moe_expert_ffn")
+    return h, y
+
+
+def combine(cfg: Config, y, slot_of, topk_w=None, weights_applied: bool = True, out=None, stream=None):
+    if out is None:
+        out = _empty((cfg.T, cfg.d), cfg.torch_dtype, y)
+    _check(lib.moe_combine(cfg.ref, _dev_ptr(y), _dev_ptr(slot_of), _dev_ptr(topk_w), int(bool(weights_applied)),
+                           _dev_ptr(out), _stream(stream, y.device)), "moe_combine")
+    return out
+
+
+def layer_forward(cfg: Config, x, w_router, w_gate, w_up, w_down, logit_bias=None, out=None, stats=None,
+                  ws=None, stream=None):
+    """The whole layer; returns out [T, d] (stats, if given, is filled on the device)."""
+    if out is None:
+        out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
+    if ws is None:
+        ws = _empty((max(workspace_size(cfg), 1),), torch.uint8, x)
+    _check(lib.moe_layer_forward(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(logit_bias), _dev_ptr(w_gate),
+                                 _dev_ptr(w_up), _dev_ptr(w_down), _dev_ptr(out), _dev_ptr(stats), _dev_ptr(ws),
+                                 ws.numel(), _stream(stream, x.device)), "moe_layer_forward")
+    return out
+
+
+def layer_forward_host(cfg: Config, x_host, w_router, w_gate, w_up, w_down, out_host, ws, logit_bias=None,
+                       stream=None):
+    """The layer with x and out in (preferably pinned) host memory; returns when out_host is filled."""
+    if x_host.is_cuda or out_host.is_cuda:
+        raise ValueError("x_host and out_host must be host tensors")
+    _check(lib.moe_layer_forward_host(cfg.ref, _ptr(x_host), _dev_ptr(w_router), _dev_ptr(logit_bias),
+                                      _dev_ptr(w_gate), _dev_ptr(w_up), _dev_ptr(w_down), _ptr(out_host),
+                                      _dev_ptr(ws), ws.numel(), _stream(stream, w_router.device)),
+           "moe_layer_forward_host")
+    return out_host
+
+
+def get_device_error(clear: bool = True) -> int:
+    code = ctypes.c_int32(0)
+    st = lib.moe_get_device_error(ctypes.byref(code), int(bool(clear)))
+    if st not in (0, 5):
+        raise MoEError(st, "moe_get_device_error")
+    return int(code.value)

@@ -1,0 +1,83 @@
+// Weighted combine back to token order.
+//
+// "How does Grok-1 use a mixture-of-experts design?", section "The high-level
+// architecture": `_dispatch_and_combine(...).view_as(x)` returns, for every
+// token, the routing-weighted sum of its experts' outputs (the page "Let Grok
+// spill the beans on Grok" names it a weighted sum); section "Expert
+// parallelism vs. tensor parallelism" scales each expert output by its weight.
+//
+// out[t] = sum_{j: slot_of[t,j] >= 0} s_j * y[slot_of[t,j]] in fp32, j = 0
+// first, then one rounding to the output type.  A fixed order and a zero start
+// make the result independent of scheduling.  HBM-bound: one block per token
+// row per iteration, 16-byte loads of y.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot_of,
+                                                     const float* __restrict__ topk_w, int weights_applied, int64_t T,
+                                                     int64_t d, int64_t max_slot, void* __restrict__ out, int* err) {
+  const int64_t nvec = d / 4;  // float4 groups per row
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const int2 sl = __ldg(reinterpret_cast<const int2*>(slot_of) + t);
+    int s0 = sl.x, s1 = sl.y;
+    if (s0 >= max_slot || s0 < -1 || s1 >= max_slot || s1 < -1) {
+      if (threadIdx.x == 0) flag_error(err, MOE_DEVERR_SLOT_INDEX);
+      if (s0 >= max_slot || s0 < -1) s0 = -1;
+      if (s1 >= max_slot || s1 < -1) s1 = -1;
+    }
+    float c0 = 1.f, c1 = 1.f;
+    if (!weights_applied) {
+      const float2 wt = __ldg(reinterpret_cast<const float2*>(topk_w) + t);
+      c0 = wt.x;
+      c1 = wt.y;
+    }
+    const float4* y0 = reinterpret_cast<const float4*>(y + (int64_t)(s0 < 0 ? 0 : s0) * d);
+    const float4* y1 = reinterpret_cast<const float4*>(y + (int64_t)(s1 < 0 ? 0 : s1) * d);
+    for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s0 >= 0) {
+        const float4 p = __ldg(y0 + v);
+        a.x += c0 * p.x; a.y += c0 * p.y; a.z += c0 * p.z; a.w += c0 * p.w;
+      }
+      if (s1 >= 0) {
+        const float4 p = __ldg(y1 + v);
+        a.x += c1 * p.x; a.y += c1 * p.y; a.z += c1 * p.z; a.w += c1 * p.w;
+      }
+      if (kBf16Out) {
+        uint2 o;
+        o.x = pack_bf16x2(a.x, a.y);
+        o.y = pack_bf16x2(a.z, a.w);
+        reinterpret_cast<uint2*>(out)[t * nvec + v] = o;
+      } else {
+        reinterpret_cast<float4*>(out)[t * nvec + v] = a;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_config_t& c, const float* y, const int32_t* slot_of,
+                           const float* topk_w, int weights_applied, void* out, cudaStream_t s,
+                           const Ctx& ctx) {
+  if (c.T == 0) return cudaSuccess;
+  int64_t blocks = c.T;
+  const int64_t cap_blocks = (int64_t)ctx.num_sms * 8;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  const int64_t max_slot = slot_rows(c);
+  if (c.dtype == MOE_BF16)
+    combine_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(y, slot_of, topk_w, weights_applied, c.T, c.d, max_slot,
+                                                          out, ctx.err);
+  else
+    combine_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(y, slot_of, topk_w, weights_applied, c.T, c.d, max_slot,
+                                                           out, ctx.err);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,397 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "How does Grok-1 use a mixture-of-experts design?", section "Expert
+// implementation: SwiGLU at scale": every expert is y = W_down(silu(W_gate x) *
+// W_up x) without bias, and FusedSwiGLUExpert computes gate and up with one
+// matmul of width 2f.  Here:
+//   gate/up : rows r of expert e:  H[r, n0:n0+128] = silu(X W_gate[e]) * (X W_up[e])
+//             one 128 x 256 x 16 MMA per K step covers the gate AND up columns
+//             of the tile (two 64-column chunks of each weight side by side in
+//             shared memory), so the SwiGLU is applied in the epilogue straight
+//             from the TMEM accumulator and H is written once, in bf16.
+//   down    : Y[r, n0:n0+BN] = row_scale[r] * (H W_down[e])   (fp32 out)
+//
+// Layouts: X / H row-major [rows, K] (K-major A); weights row-major [E, K, N]
+// (N contiguous, so B is MN-major, legal for 16-bit UMMA).  One TMA box per
+// 128 B x 64 rows, 128-byte swizzle on both sides.
+//
+// Schedule: persistent, one CTA per SM.  The tile list is every
+// (expert, 128-row block, N block); tiles of one expert are ordered N-block
+// major so CTAs running at the same time share weight tiles and row blocks in
+// L2.  Rows of an expert's last block that belong to the next expert are
+// computed but not stored.  Warp roles (192 threads):
+//   warp 0 lane 0 : TMA producer over a kStages ring (full/empty mbarriers)
+//   warp 1 lane 0 : MMA issuer; warp 1 owns the 512 TMEM columns
+//                   (two 256-column fp32 accumulators, double buffered)
+//   warps 2..5    : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+// Every mbarrier wait is bounded; on a timeout the CTA flags the device error
+// word, the other roles stop, in-flight copies and MMAs are drained and TMEM is
+// released before the CTA exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+using namespace ptx;
+
+constexpr int kE = 8;
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kAccStride = 256;  // TMEM columns between the two accumulators
+constexpr int A_BYTES = BM * BK * 2;      // 16 KB
+constexpr int CHUNK_BYTES = 64 * BK * 2;  // 8 KB: 64 N-columns x 64 K-rows
+
+enum Mode { kGateUp = 0, kDown = 1 };
+
+template <int MODE, int MMA_N>
+struct Cfg {
+  static constexpr int kChunks = MMA_N / 64;
+  static constexpr int B_BYTES = kChunks * CHUNK_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int kStages = MMA_N == 256 ? 4 : 6;
+  static constexpr int BN_OUT = MODE == kGateUp ? MMA_N / 2 : MMA_N;  // output columns per tile
+  static constexpr int kBarBytes = 256;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + kBarBytes;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N, false, true);
+};
+
+struct TcArgs {
+  const int32_t* offsets;  // [E + 1], device
+  int64_t rows_alloc;      // rows of the A and output buffers
+  int n_tiles;             // output N / BN_OUT
+  int num_kb;              // K / BK
+  void* out;
+  int64_t ld_out;          // elements per output row
+  const float* row_scale;  // down only; NULL means 1
+  int* err;
+};
+
+struct Sched {
+  int offs[kE + 1];
+  int mt[kE];
+  int prefix[kE + 1];
+};
+
+struct Tile {
+  int e, m0, rows, n0;
+};
+
+__device__ __forceinline__ Tile decode_tile(const Sched& s, int L, int bn) {
+  int e = 0;
+#pragma unroll
+  for (int k = 1; k < kE; ++k)
+    if (L >= s.prefix[k]) e = k;
+  const int local = L - s.prefix[e];
+  const int nt = local / s.mt[e];
+  const int mi = local - nt * s.mt[e];
+  Tile t;
+  t.e = e;
+  t.m0 = s.offs[e] + mi * BM;
+  const int left = s.offs[e + 1] - t.m0;
+  t.rows = left < BM ? left : BM;
+  t.n0 = nt * bn;
+  return t;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+template <int MODE, int MMA_N>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                           const __grid_constant__ CUtensorMap tmB1, const TcArgs args) {
+  using C = Cfg<MODE, MMA_N>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ Sched sched;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 1) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB0);
+    prefetch_tmap(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 2 && lane == 0) {
+    bool ok = true;
+    int prev = 0;
+    for (int k = 0; k <= kE; ++k) {
+      const int v = args.offsets[k];
+      sched.offs[k] = v;
+      if (v < prev || (int64_t)v > args.rows_alloc) ok = false;
+      prev = v;
+    }
+    if (sched.offs[0] < 0) ok = false;
+    int acc = 0;
+    for (int k = 0; k < kE; ++k) {
+      const int n = ok ? sched.offs[k + 1] - sched.offs[k] : 0;
+      sched.mt[k] = (n + BM - 1) / BM;
+      sched.prefix[k] = acc;
+      acc += sched.mt[k] * args.n_tiles;
+    }
+    sched.prefix[kE] = acc;
+    if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = sched.prefix[kE];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        const Tile t = decode_tile(sched, L, C::BN_OUT);
+        for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          uint8_t* b = sB + s * C::B_BYTES;
+          tma_load_2d(sA + s * A_BYTES, &tmA, &full[s], kb * BK, t.m0);
+          if (MODE == kGateUp) {
+#pragma unroll
+            for (int c = 0; c < C::kChunks / 2; ++c) {
+              tma_load_3d(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e);
+              tma_load_3d(b + (C::kChunks / 2 + c) * CHUNK_BYTES, &tmB1, &full[s], t.n0 + 64 * c, kb * BK, t.e);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e);
+          }
+        }
+      }
+      if (!ok) {
+        flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // drain: every issued load must land before the CTA can exit
+      const uint32_t first = it > (uint32_t)S ? it - S : 0u;
+      for (uint32_t j = first; j < it; ++j) mbar_wait(&full[j % S], (j / S) & 1u, nullptr, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t it = 0, tc = 0;
+      bool ok = true, issued = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        const uint32_t buf = tc & 1u;
+        const uint32_t tph = (tc >> 1) & 1u;
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * kAccStride;
+        for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sw128_desc(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(b_addr + kk * 2048, CHUNK_BYTES, 1024);
+            umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (issued) {
+        // all MMAs must finish before TMEM and shared memory are released
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, 100000000ull);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    uint32_t tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      const Tile t = decode_tile(sched, L, C::BN_OUT);
+      const uint32_t buf = tc & 1u;
+      const uint32_t tph = (tc >> 1) & 1u;
+      if (!mbar_wait(&tfull[buf], tph, abort_flag)) {
+        if (lane == 0) flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const bool valid = r < t.rows;
+      const uint32_t tacc = tmem_base + buf * kAccStride + ((uint32_t)(q * 32) << 16);
+      if (MODE == kGateUp) {
+        __nv_bfloat16* H = static_cast<__nv_bfloat16*>(args.out);
+        __nv_bfloat16* dst_row = H + (int64_t)(t.m0 + r) * args.ld_out + t.n0;
+#pragma unroll 1
+        for (int c = 0; c < C::BN_OUT / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tacc + c * 32, g);
+          tmem_ld32(tacc + C::BN_OUT + c * 32, u);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            p[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                               silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else {
+        float* Y = static_cast<float*>(args.out);
+        float* dst_row = Y + (int64_t)(t.m0 + r) * args.ld_out + t.n0;
+        const float sc = (valid && args.row_scale) ? __ldg(args.row_scale + t.m0 + r) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < C::BN_OUT / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(dst_row + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(sc * __uint_as_float(v[4 * i]), sc * __uint_as_float(v[4 * i + 1]),
+                                  sc * __uint_as_float(v[4 * i + 2]), sc * __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int MODE, int MMA_N>
+cudaError_t launch_grouped(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const TcArgs& args,
+                           cudaStream_t s, const Ctx& ctx) {
+  using C = Cfg<MODE, MMA_N>;
+  auto kern = grouped_gemm_tc_kernel<MODE, MMA_N>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<ctx.num_sms, kThreads, C::SMEM_BYTES, s>>>(a, b0, b1, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
+                              const void* wg, const void* wu, void* h, cudaStream_t s, const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap ta, tg, tu;
+  const uint64_t a_dims[2] = {(uint64_t)c.d, (uint64_t)rows};
+  const uint64_t a_str[1] = {(uint64_t)c.d * 2};
+  const uint32_t a_box[2] = {64, 128};
+  const uint64_t w_dims[3] = {(uint64_t)c.f, (uint64_t)c.d, (uint64_t)c.E};
+  const uint64_t w_str[2] = {(uint64_t)c.f * 2, (uint64_t)c.d * c.f * 2};
+  const uint32_t w_box[3] = {64, 64, 1};
+  if (!encode_tmap(&ta, x_perm, 2, a_dims, a_str, a_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tg, wg, 3, w_dims, w_str, w_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tu, wu, 3, w_dims, w_str, w_box, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  TcArgs args;
+  args.offsets = offsets;
+  args.rows_alloc = rows;
+  args.n_tiles = (int)(c.f / Cfg<kGateUp, 256>::BN_OUT);
+  args.num_kb = (int)(c.d / BK);
+  args.out = h;
+  args.ld_out = c.f;
+  args.row_scale = nullptr;
+  args.err = ctx.err;
+  return launch_grouped<kGateUp, 256>(ta, tg, tu, args, s, ctx);
+}
+
+cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
+                           const float* row_scale, float* y, cudaStream_t s, const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap ta, tw;
+  const uint64_t a_dims[2] = {(uint64_t)c.f, (uint64_t)rows};
+  const uint64_t a_str[1] = {(uint64_t)c.f * 2};
+  const uint32_t a_box[2] = {64, 128};
+  const uint64_t w_dims[3] = {(uint64_t)c.d, (uint64_t)c.f, (uint64_t)c.E};
+  const uint64_t w_str[2] = {(uint64_t)c.d * 2, (uint64_t)c.f * c.d * 2};
+  const uint32_t w_box[3] = {64, 64, 1};
+  if (!encode_tmap(&ta, h, 2, a_dims, a_str, a_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tw, wd, 3, w_dims, w_str, w_box, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  TcArgs args;
+  args.offsets = offsets;
+  args.rows_alloc = rows;
+  args.num_kb = (int)(c.f / BK);
+  args.out = y;
+  args.ld_out = c.d;
+  args.row_scale = row_scale;
+  args.err = ctx.err;
+  if (c.d % 256 == 0) {
+    args.n_tiles = (int)(c.d / 256);
+    return launch_grouped<kDown, 256>(ta, tw, tw, args, s, ctx);
+  }
+  args.n_tiles = (int)(c.d / 128);
+  return launch_grouped<kDown, 128>(ta, tw, tw, args, s, ctx);
+}
+
+}  // namespace moe

@@ -1,0 +1,380 @@
+// C ABI of libmoe_b200: argument checks, workspace layout and the launch
+// sequence of the MoE layer forward pass.  Every compute step runs in the
+// kernels of this library; this file only validates and enqueues.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+// Device error word (MOE_DEVERR_* bits), one per device that loads the library.
+__device__ int g_moe_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+Ctx g_ctx[kMaxDevices];
+std::mutex g_ctx_mu;
+
+moe_status_t get_ctx(Ctx& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_ctx_mu);
+  Ctx& c = g_ctx[dev];
+  if (c.dev != dev) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_device_error) != cudaSuccess) return MOE_ERR_CUDA;
+    c.num_sms = sms;
+    c.err = static_cast<int*>(p);
+    c.dev = dev;
+  }
+  out = c;
+  return MOE_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t esize(const moe_config_t& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+
+moe_status_t check_config(const moe_config_t* cfg) {
+  if (!cfg) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  if (c.T < 0 || c.d <= 0 || c.f <= 0 || c.reserved != 0) return MOE_ERR_INVALID_ARG;
+  if (!(c.capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;  // rejects NaN too
+  if (c.dtype != MOE_F32 && c.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c.E != 8 || c.top_k != 2) return MOE_ERR_UNSUPPORTED;
+  if (c.T > (int64_t)1 << 24 || c.d > (int64_t)1 << 20 || c.f > (int64_t)1 << 20) return MOE_ERR_UNSUPPORTED;
+  const int64_t mult = c.dtype == MOE_BF16 ? 128 : 64;
+  if (c.d % mult != 0 || c.f % mult != 0) return MOE_ERR_UNSUPPORTED;
+  if (c.dtype == MOE_F32 && (slot_rows(c) + 63) / 64 + 8 > 65535) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// ceil(cf * T * k / E) in double, in that order; never more than T, which no
+// expert can exceed anyway (a token reaches an expert at most once).
+int64_t capacity_of(const moe_config_t& c) {
+  if (isinf(c.capacity_factor)) return c.T;
+  const double v = ceil(c.capacity_factor * (double)(c.T * c.top_k) / (double)c.E);
+  if (v >= (double)c.T) return c.T;
+  return (int64_t)v;
+}
+
+size_t round_up(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Scratch of moe_dispatch: per-block expert histograms.
+size_t dispatch_ws(const moe_config_t& c) { return round_up((size_t)dispatch_blocks(c) * c.E * sizeof(int32_t)); }
+
+// Workspace of moe_layer_forward, carved in this order.
+struct Layout {
+  size_t topk_idx, topk_w, route, perm, slot_of, row_scale, disp, x_perm, h, y, x_in, out, total;
+};
+
+Layout layout_of(const moe_config_t& c) {
+  Layout L;
+  const size_t rows = (size_t)slot_rows(c);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += round_up(bytes);
+    return at;
+  };
+  L.topk_idx = take(rows * 4);
+  L.topk_w = take(rows * 4);
+  L.route = take((size_t)(3 * c.E + 2 + 8) * 4);  // counts_raw, counts_kept, offsets, stats
+  L.perm = take(rows * 4);
+  L.slot_of = take(rows * 4);
+  L.row_scale = take(rows * 4);
+  L.disp = take(dispatch_ws(c));
+  L.x_perm = take(rows * c.d * esize(c));
+  L.h = take(rows * c.f * esize(c));
+  L.y = take(rows * c.d * 4);
+  L.x_in = take((size_t)c.T * c.d * esize(c));
+  L.out = take((size_t)c.T * c.d * esize(c));
+  L.total = o;
+  return L;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status_t run_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets, const void* wg,
+                         const void* wu, void* h, cudaStream_t s, const Ctx& ctx) {
+  if (c.dtype == MOE_BF16) return cuda_status(launch_tc_gate_up(c, x_perm, offsets, wg, wu, h, s, ctx));
+  return cuda_status(launch_ffn_simt_gate_up(c, static_cast<const float*>(x_perm), offsets,
+                                             static_cast<const float*>(wg), static_cast<const float*>(wu),
+                                             static_cast<float*>(h), s, ctx));
+}
+
+moe_status_t run_down(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
+                      const float* row_scale, float* y, cudaStream_t s, const Ctx& ctx) {
+  if (c.dtype == MOE_BF16) return cuda_status(launch_tc_down(c, h, offsets, wd, row_scale, y, s, ctx));
+  return cuda_status(launch_ffn_simt_down(c, static_cast<const float*>(h), offsets, static_cast<const float*>(wd),
+                                          row_scale, y, s, ctx));
+}
+
+}  // namespace
+
+bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                 const uint32_t* box, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int64_t moe_capacity(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return -1;
+  return capacity_of(*cfg);
+}
+
+size_t moe_dispatch_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return dispatch_ws(*cfg);
+}
+
+size_t moe_expert_ffn_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return 0;
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg).total;
+}
+
+moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
+                             float* logits, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+      (logits && !aligned16(logits)) || (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return cuda_status(launch_router(*cfg, x, w_router, logit_bias, logits, topk_idx, topk_w, stream, ctx));
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const float* topk_w,
+                          int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                          float* row_scale, void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!topk_idx || !topk_w || !counts_raw || !counts_kept || !offsets || !perm || !slot_of || !row_scale)
+    return MOE_ERR_INVALID_ARG;
+  if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(slot_of) || (x_perm && !aligned16(x_perm)) ||
+      (x && !aligned16(x)))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < dispatch_ws(*cfg) || (dispatch_ws(*cfg) > 0 && !ws)) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  cudaError_t e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, counts_raw, counts_kept, offsets, perm,
+                                  slot_of, row_scale, static_cast<int32_t*>(ws), nullptr, stream, ctx);
+  if (e == cudaSuccess && x_perm && c.T > 0) e = launch_gather(c, x, perm, offsets, x_perm, stream, ctx);
+  return cuda_status(e);
+}
+
+moe_status_t moe_expert_gate_up(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                                const void* w_gate, const void* w_up, void* h, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return run_gate_up(*cfg, x_perm, offsets, w_gate, w_up, h, stream, ctx);
+}
+
+moe_status_t moe_expert_down(const moe_config_t* cfg, const void* h, const int32_t* offsets, const void* w_down,
+                             const float* row_scale, float* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!h || !offsets || !w_down || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return run_down(*cfg, h, offsets, w_down, row_scale, y, stream, ctx);
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate,
+                            const void* w_up, const void* w_down, const float* row_scale, void* h, float* y, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = moe_expert_gate_up(cfg, x_perm, offsets, w_gate, w_up, h, stream);
+  if (st != MOE_OK) return st;
+  return moe_expert_down(cfg, h, offsets, w_down, row_scale, y, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const float* y, const int32_t* slot_of, const float* topk_w,
+                         int32_t weights_applied, void* out, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y || !slot_of || !out || (!weights_applied && !topk_w)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(slot_of) || !aligned16(out) || (topk_w && !aligned16(topk_w)))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return cuda_status(launch_combine(*cfg, y, slot_of, topk_w, weights_applied, out, stream, ctx));
+}
+
+static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, const void* w_router,
+                                       const float* logit_bias, const void* w_gate, const void* w_up,
+                                       const void* w_down, void* out, int32_t* stats, uint8_t* ws, cudaStream_t s,
+                                       const Ctx& ctx) {
+  const Layout L = layout_of(c);
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  int32_t* route = reinterpret_cast<int32_t*>(ws + L.route);
+  int32_t* counts_raw = route;
+  int32_t* counts_kept = route + c.E;
+  int32_t* offsets = route + 2 * c.E;
+  int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
+  float* row_scale = reinterpret_cast<float*>(ws + L.row_scale);
+  int32_t* disp = reinterpret_cast<int32_t*>(ws + L.disp);
+  void* x_perm = ws + L.x_perm;
+  void* h = ws + L.h;
+  float* y = reinterpret_cast<float*>(ws + L.y);
+
+  cudaError_t e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, s, ctx);
+  if (e == cudaSuccess)
+    e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, counts_raw, counts_kept, offsets, perm, slot_of,
+                        row_scale, disp, stats, s, ctx);
+  if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, x_perm, s, ctx);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  moe_status_t st = run_gate_up(c, x_perm, offsets, w_gate, w_up, h, s, ctx);
+  if (st == MOE_OK) st = run_down(c, h, offsets, w_down, row_scale, y, s, ctx);
+  if (st == MOE_OK) st = cuda_status(launch_combine(c, y, slot_of, topk_w, 1, out, s, ctx));
+  return st;
+}
+
+static moe_status_t check_layer_args(const moe_config_t* cfg, const void* w_router, const float* logit_bias,
+                                     const void* w_gate, const void* w_up, const void* w_down, void* ws,
+                                     size_t ws_bytes) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!w_router || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!ws || ws_bytes < layout_of(*cfg).total)) return MOE_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
+                               const void* w_gate, const void* w_up, const void* w_down, void* out, int32_t* stats,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out) || (stats && !aligned16(stats))) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return layer_forward_impl(*cfg, x, w_router, logit_bias, w_gate, w_up, w_down, out, stats,
+                            static_cast<uint8_t*>(ws), stream, ctx);
+}
+
+moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host, const void* w_router,
+                                    const float* logit_bias, const void* w_gate, const void* w_up, const void* w_down,
+                                    void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  const Layout L = layout_of(c);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const size_t bytes = (size_t)c.T * c.d * esize(c);
+  if (cudaMemcpyAsync(w8 + L.x_in, x_host, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = layer_forward_impl(c, w8 + L.x_in, w_router, logit_bias, w_gate, w_up, w_down, w8 + L.out, nullptr, w8,
+                          stream, ctx);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, w8 + L.out, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(stream));
+}
+
+moe_status_t moe_get_device_error(int32_t* code, int32_t clear) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  moe_status_t st = get_ctx(ctx);
+  if (st != MOE_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ctx.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpy(ctx.err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  *code = v;
+  return v ? MOE_ERR_DEVICE_CHECK : MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects bad arguments before touching the device."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from sparse_moe_layer_07_b200 import build
+
+    build.build()
+    import sparse_moe_layer_07_b200 as m
+
+    return m
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = declared_symbols()
+    for n in ("moe_router_topk", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(moe):
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def _cfg(moe, **kw):
+    base = dict(T=64, d=256, f=1024, capacity_factor=1.25, dtype="f32")
+    base.update(kw)
+    return moe.Config(**base)
+
+
+def test_status_strings(moe):
+    for code, name in moe.STATUS.items():
+        assert moe.lib.moe_status_string(code).decode() == name
+
+
+def test_capacity_matches_oracle(moe):
+    import oracle
+
+    for T, cf in [(64, 1.25), (2048, 1.25), (8192, 4.0), (16384, 1.25), (10, 1.0), (7, 0.3), (32, math.inf),
+                  (100, 1.1), (1000, 0.01), (5, 100.0)]:
+        c = _cfg(moe, T=T, capacity_factor=cf)
+        assert moe.capacity(c) == min(oracle.capacity(T, 2, 8, cf), T), (T, cf)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(E=4), "MOE_ERR_UNSUPPORTED"),
+    (dict(top_k=1), "MOE_ERR_UNSUPPORTED"),
+    (dict(d=100), "MOE_ERR_UNSUPPORTED"),
+    (dict(dtype="bf16", f=192), "MOE_ERR_UNSUPPORTED"),
+    (dict(capacity_factor=0.0), "MOE_ERR_INVALID_ARG"),
+    (dict(capacity_factor=float("nan")), "MOE_ERR_INVALID_ARG"),
+    (dict(capacity_factor=-1.0), "MOE_ERR_INVALID_ARG"),
+    (dict(T=-1), "MOE_ERR_INVALID_ARG"),
+])
+def test_bad_config_rejected_before_launch(moe, kw, status):
+    c = _cfg(moe, **kw)
+    P = ctypes.c_void_p
+    fake = P(16)  # never dereferenced: validation fails first
+    st = moe.lib.moe_router_topk(c.ref, fake, fake, None, None, fake, fake, None)
+    assert moe.STATUS[st] == status
+    assert moe.capacity(c) == -1
+    assert moe.workspace_size(c) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(moe):
+    c = _cfg(moe)
+    P = ctypes.c_void_p
+    ok = P(256)
+    assert moe.STATUS[moe.lib.moe_router_topk(c.ref, None, ok, None, None, ok, ok, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[moe.lib.moe_router_topk(c.ref, P(258), ok, None, None, ok, ok, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[moe.lib.moe_combine(c.ref, ok, ok, None, 0, ok, None)] == "MOE_ERR_INVALID_ARG"
+    st = moe.lib.moe_layer_forward(c.ref, ok, None, None, ok, ok, ok, ok, None, ok, 1 << 30, None)
+    assert moe.STATUS[st] == "MOE_ERR_INVALID_ARG"
+
+
+def test_small_workspace_rejected(moe):
+    c = _cfg(moe, T=4096)
+    P = ctypes.c_void_p
+    ok = P(256)
+    need = moe.dispatch_workspace_size(c)
+    assert need >= 16 * 8 * 4
+    st = moe.lib.moe_dispatch(c.ref, ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, need - 1, None)
+    assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
+    st = moe.lib.moe_layer_forward(c.ref, ok, ok, None, ok, ok, ok, ok, None, ok, moe.workspace_size(c) - 1, None)
+    assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
+
+
+def test_empty_batch_is_a_no_op(moe):
+    c = _cfg(moe, T=0)
+    P = ctypes.c_void_p
+    ok = P(256)
+    assert moe.lib.moe_router_topk(c.ref, None, None, None, None, None, None, None) == 0
+    assert moe.lib.moe_layer_forward(c.ref, None, ok, None, ok, ok, ok, None, None, None, 0, None) == 0
+
+
+def test_workspace_grows_with_tokens(moe):
+    a = moe.workspace_size(_cfg(moe, T=64, dtype="bf16"))
+    b = moe.workspace_size(_cfg(moe, T=128, dtype="bf16"))
+    assert 0 < a < b
