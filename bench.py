@@ -66,7 +66,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
@@ -161,7 +161,7 @@ def workload_config(w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="grok_prefill", choices=sorted(configs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -170,8 +170,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--shape", default=None, help="T,d,f override of the workload (profiling cases)")
     args = ap.parse_args()
     w = configs.WORKLOADS[args.workload]
+    if args.shape:
+        T, d, f = (int(v) for v in args.shape.split(","))
+        w = configs.scaled(w, name=f"{w.name}_T{T}_d{d}_f{f}", T=T, d=d, f=f)
     if args.impl == "reference":
         return reference_arm(args, w)
 
@@ -352,7 +356,7 @@ def main():
         del ws_full
 
     # ---- decode (weight streaming) on the same Grok-shape weights
-    if not args.no_decode and w.name == "grok_prefill":
+    if not args.no_decode and w.name == "grok_prefill" and not args.shape:
         line["decode"] = decode_bench(moe, W, dev, stream, peaks, peak_src, world)
 
     if rank == 0 and world == 1 and not args.no_cpu and host is not None:

@@ -14,8 +14,8 @@ import oracle
 import sparse_moe_layer_07_b200 as moe
 from synth import configs
 
-from parity_util import (LayerInputs, check_dispatch, check_out_rows, check_routing, run_steps, to_dev,
-                         to_np64)
+from parity_util import (LayerInputs, check_dispatch, check_layer_out, check_out_rows, check_routing,
+                         run_steps, to_dev, to_np64)
 
 pytestmark = pytest.mark.gpu
 
@@ -97,8 +97,10 @@ def test_hidden_and_expert_outputs(case):
 def test_layer_output(case):
     L, g, ref = case
     got = to_np64(g["out"])
-    rows = np.nonzero((np.sort(g["idx"], 1) == np.sort(ref["idx"], 1)).all(1))[0]
-    check_out_rows(L, got[rows], ref["out"][rows], L.w.storage)
+    same_route = (np.sort(g["idx"], 1) == np.sort(ref["idx"], 1)).all(1)
+    same_keep = ((g["slot_of"] >= 0) == (ref["slot_of"] >= 0)).all(1) | ~same_route
+    rows = np.nonzero(same_route & same_keep)[0]
+    check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"][rows], rows)
     # tokens whose assignments were all dropped output exactly zero
     dropped = (g["slot_of"] < 0).all(axis=1)
     assert np.all(got[dropped] == 0.0)
@@ -157,7 +159,7 @@ def test_all_tokens_to_two_experts_drop_and_zero():
     assert (g["slot_of"][cap:] == -1).all()
     assert np.all(to_np64(g["out"])[cap:] == 0.0)
     ref = oracle.layer_forward(L.x, L.wr, L.wg, L.wu, L.wd, w.capacity_factor, logit_bias=L.bias)
-    check_out_rows(L, to_np64(g["out"]), ref["out"], "bf16")
+    check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"], np.arange(256))
 
 
 def test_bad_expert_index_sets_device_error_without_trap():
