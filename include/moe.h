@@ -197,6 +197,29 @@ MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void*
                                     const void* w_down, void* out_host, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
 
+/* Largest T accepted by moe_dispatch_noalloc. */
+#define MOE_NOALLOC_MAX_TOKENS (1 << 20)
+
+/* moe_dispatch without a caller-provided workspace and without allocating,
+ * for callers that cannot allocate device memory: plug-ins hosted by a runtime
+ * that owns all device memory and gives them no workspace, and latency-critical
+ * loops that cannot afford cudaMalloc's implicit device-wide synchronisation.
+ * The pages have no counterpart to this entry point (it concerns memory
+ * management only); it computes exactly what moe_dispatch computes, with the
+ * same arguments minus ws/ws_bytes.
+ * Its scratch (per-block expert histograms) is a fixed device array inside
+ * the library, 128 KiB held by every GPU that loads the library until the
+ * process exits.  T > MOE_NOALLOC_MAX_TOKENS returns MOE_ERR_UNSUPPORTED.  All
+ * calls share that array: calls that overlap on the GPU (e.g. on two streams)
+ * race.  The array keeps the last call's contents; each call writes every
+ * entry it reads, so nothing needs clearing.  The first call on a device looks
+ * up the array's device address with that device current; make it before any
+ * stream capture.  No cudaMalloc, cudaFree or allocating routine is called. */
+MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                          const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
+                                          int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                                          float* row_scale, void* x_perm, moe_stream_t stream);
+
 /* Waits for the current device, returns the device error word (MOE_DEVERR_*
  * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.
  * Returns MOE_ERR_DEVICE_CHECK when the word is non-zero, else MOE_OK. */

@@ -21,7 +21,7 @@ __all__ = [
     "MoEError", "Config", "LIB_PATH", "lib", "abi_version", "capacity", "workspace_size",
     "dispatch_workspace_size", "router_topk", "dispatch", "expert_ffn", "expert_gate_up",
     "expert_down", "combine", "layer_forward", "layer_forward_host", "get_device_error",
-    "STATUS", "DEVERR",
+    "STATUS", "DEVERR", "dispatch_noalloc", "NOALLOC_MAX_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -30,6 +30,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 DEVERR = {"EXPERT_INDEX": 0x1, "SLOT_INDEX": 0x2, "OFFSETS": 0x4, "TIMEOUT": 0x8}
 _DTYPES = {"f32": 0, "bf16": 1}
+NOALLOC_MAX_TOKENS = 1 << 20
 _TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
@@ -69,6 +70,7 @@ def _load():
         "moe_layer_forward": ([cfgp, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_host": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32], ctypes.c_int),
+        "moe_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -190,6 +192,30 @@ def dispatch(cfg: Config, x, topk_idx, topk_w, gather: bool = True, out=None, ws
                             _dev_ptr(o["counts_kept"]), _dev_ptr(o["offsets"]), _dev_ptr(o["perm"]),
                             _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]), _dev_ptr(o["x_perm"]),
                             _dev_ptr(ws), ws.numel(), _stream(stream, dev.device)), "moe_dispatch")
+    return o
+
+
+def dispatch_noalloc(cfg: Config, x, topk_idx, topk_w, gather: bool = True, out=None, stream=None):
+    """moe_dispatch_noalloc: the same outputs as dispatch(), with the library's own fixed
+    scratch instead of a caller workspace (for callers that cannot allocate device memory).
+    Output tensors are allocated here only when the caller does not pass them in `out`."""
+    dev = topk_idx
+    rows = cfg.T * cfg.top_k
+    o = dict(out or {})
+    o.setdefault("counts_raw", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("counts_kept", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("offsets", _empty((cfg.E + 1,), torch.int32, dev))
+    o.setdefault("perm", _empty((rows,), torch.int32, dev))
+    o.setdefault("slot_of", _empty((cfg.T, cfg.top_k), torch.int32, dev))
+    o.setdefault("row_scale", _empty((rows,), torch.float32, dev))
+    if gather:
+        o.setdefault("x_perm", _empty((rows, cfg.d), cfg.torch_dtype, dev))
+    else:
+        o["x_perm"] = None
+    _check(lib.moe_dispatch_noalloc(cfg.ref, _dev_ptr(x), _dev_ptr(topk_idx), _dev_ptr(topk_w),
+                                    _dev_ptr(o["counts_raw"]), _dev_ptr(o["counts_kept"]), _dev_ptr(o["offsets"]),
+                                    _dev_ptr(o["perm"]), _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]),
+                                    _dev_ptr(o["x_perm"]), _stream(stream, dev.device)), "moe_dispatch_noalloc")
     return o
 
 

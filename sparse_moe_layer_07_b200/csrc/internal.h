@@ -56,6 +56,11 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
                            const void* wd, const float* row_scale, float* y, cudaStream_t s,
                            const Ctx& ctx);
 
+// Argument check shared by the entry points (MOE_OK when the config is usable).
+moe_status_t validate_config(const moe_config_t* cfg);
+// Device facts of the current device (cached per device).
+moe_status_t current_ctx(Ctx& out);
+
 // Encodes a tiled TMA descriptor (driver entry point resolved once).
 bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz);

@@ -139,6 +139,10 @@ moe_status_t run_down(const moe_config_t& c, const void* h, const int32_t* offse
 
 }  // namespace
 
+moe_status_t validate_config(const moe_config_t* cfg) { return check_config(cfg); }
+
+moe_status_t current_ctx(Ctx& out) { return get_ctx(out); }
+
 bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                  const uint32_t* box, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();

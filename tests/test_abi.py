@@ -113,3 +113,17 @@ def test_workspace_grows_with_tokens(moe):
     a = moe.workspace_size(_cfg(moe, T=64, dtype="bf16"))
     b = moe.workspace_size(_cfg(moe, T=128, dtype="bf16"))
     assert 0 < a < b
+
+
+def test_noalloc_dispatch_rejects_oversize_before_launch(moe):
+    P = ctypes.c_void_p
+    ok = P(256)
+    big = _cfg(moe, T=moe.NOALLOC_MAX_TOKENS + 1, dtype="bf16", d=256, f=384)
+    st = moe.lib.moe_dispatch_noalloc(big.ref, None, ok, ok, ok, ok, ok, ok, ok, ok, None, None)
+    assert moe.STATUS[st] == "MOE_ERR_UNSUPPORTED"
+    bad = _cfg(moe, E=4)
+    assert moe.STATUS[moe.lib.moe_dispatch_noalloc(bad.ref, None, ok, ok, ok, ok, ok, ok, ok, ok, None,
+                                                   None)] == "MOE_ERR_UNSUPPORTED"
+    small = _cfg(moe, T=64)
+    assert moe.STATUS[moe.lib.moe_dispatch_noalloc(small.ref, None, None, ok, ok, ok, ok, ok, ok, ok, None,
+                                                   None)] == "MOE_ERR_INVALID_ARG"
