@@ -42,11 +42,78 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_tc_dram_grok_prefill_T8192_d6144_f32768.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_07_b200", "csrc", n) for n in ("ffn_tc.cu", "tc_ptx.cuh")]
+
+
+def measured_traffic(workload_name):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary,
+    or None when the workload differs or the kernel sources changed since the capture."""
+    import hashlib
+
+    if workload_name != "grok_prefill" or not os.path.exists(TRAFFIC_FILE):
+        return None
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    fields = {}
+    with open(TRAFFIC_FILE) as fh:
+        for line in fh:
+            if ":" in line:
+                k, v = line.strip().split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_sources_sha256") != h.hexdigest():
+        return None
+    try:
+        return float(fields["gate_up_dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+# ---------------------------------------------------------------------------- multi-rank plumbing
+def rank_x(w, rank):
+    """The batch of rank `rank`: rank 0 runs the workload's own x; rank r > 0 a distinct
+    seeded batch of the same shape (independent token batches, no exchange)."""
+    if rank == 0:
+        return configs.make_x(w)
+    from synth import normal
+
+    return normal(configs.SEED, configs.TID_X + 1000 * rank, (w.T, w.d), dtype=w.storage)
+
+
+def share_weights(W, world):
+    """Rank 0 generated the weights; every other rank receives them once at set-up."""
+    import torch.distributed as dist
+
+    if world > 1:
+        for k in sorted(W):
+            dist.broadcast(W[k], src=0)
+    return W
+
+
+def max_over_ranks(value, device, world):
+    """The slowest rank's time (every rank gets the same number)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world, tokens_per_rank_step, steps, ms_total):
+    """Whole-job tokens/s: the tokens of all ranks over the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (ms_total / 1000.0)
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -208,13 +275,8 @@ def main():
              "wg": torch.empty((w.E, w.d, w.f), dtype=tdt, device=dev),
              "wu": torch.empty((w.E, w.d, w.f), dtype=tdt, device=dev),
              "wd": torch.empty((w.E, w.f, w.d), dtype=tdt, device=dev)}
-    if world > 1:
-        for k in ("wr", "wg", "wu", "wd"):
-            dist.broadcast(W[k], src=0)
-    from synth import normal
-
-    x_np = configs.make_x(w) if rank == 0 else normal(configs.SEED, configs.TID_X + 1000 * rank, (w.T, w.d),
-                                                       dtype=w.storage)
+    share_weights(W, world)
+    x_np = rank_x(w, rank)
     x = to_dev(x_np)
     bias = configs.make_bias(w)
     bias_d = None if bias is None else to_dev(bias)
@@ -293,13 +355,10 @@ def main():
         for j, n in enumerate(names):
             per_kernel[n] += e[j].elapsed_time(e[j + 1])
     per_kernel = {n: v / args.steps for n, v in per_kernel.items()}
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev, world)
     ms_step = ms_total / args.steps
     tokens = world * w.T * args.steps
-    value = tokens / (ms_total / 1000.0)
+    value = throughput(world, w.T, args.steps, ms_total)
     flops_step = 2.0 * w.T * w.d * w.E + 6.0 * n_kept * w.d * w.f
     tflops = world * flops_step * args.steps / (ms_total / 1000.0) / 1e12
 
@@ -311,7 +370,8 @@ def main():
     roofline = {"bound": "tensor", "kernel": "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
-                "traffic": None,
+                "traffic": measured_traffic(w.name),
+                "traffic_unit": "bytes per launch (dram read + write, ncu)",
                 "algorithmic": f"4*d*f*N_kept = {gu_flops:.4e} FLOP per launch (N_kept={n_kept})",
                 "down": {"achieved": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12,
                          "frac": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12 / peak}}
@@ -344,11 +404,7 @@ def main():
                                    logit_bias=bias_d)
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev, world)
         nbytes = w.T * w.d * (2 if w.storage == "bf16" else 4)
         line["e2e"] = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
                        "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms / args.steps,

@@ -83,7 +83,7 @@ struct Tile {
   int e, m0, rows, n0;
 };
 
-__device__ __forceinline__ Tile decode_tile(const Sched& s, int L, int bn) {
+__device__ __forceinline__ Tile decode_tile(const Sched& s, int L, int bn, int bm = BM) {
   int e = 0;
 #pragma unroll
   for (int k = 1; k < kE; ++k)
@@ -93,11 +93,34 @@ __device__ __forceinline__ Tile decode_tile(const Sched& s, int L, int bn) {
   const int mi = local - nt * s.mt[e];
   Tile t;
   t.e = e;
-  t.m0 = s.offs[e] + mi * BM;
+  t.m0 = s.offs[e] + mi * bm;
   const int left = s.offs[e + 1] - t.m0;
-  t.rows = left < BM ? left : BM;
+  t.rows = left < bm ? left : bm;
   t.n0 = nt * bn;
   return t;
+}
+
+// Reads and checks the expert offsets, then lays out the tile list: expert e
+// has ceil(rows_e / bm) row blocks times n_tiles column blocks.
+__device__ __forceinline__ void build_schedule(Sched& sched, const TcArgs& args, int bm) {
+  bool ok = true;
+  int prev = 0;
+  for (int k = 0; k <= kE; ++k) {
+    const int v = args.offsets[k];
+    sched.offs[k] = v;
+    if (v < prev || (int64_t)v > args.rows_alloc) ok = false;
+    prev = v;
+  }
+  if (sched.offs[0] < 0) ok = false;
+  int acc = 0;
+  for (int k = 0; k < kE; ++k) {
+    const int n = ok ? sched.offs[k + 1] - sched.offs[k] : 0;
+    sched.mt[k] = (n + bm - 1) / bm;
+    sched.prefix[k] = acc;
+    acc += sched.mt[k] * args.n_tiles;
+  }
+  sched.prefix[kE] = acc;
+  if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
@@ -148,26 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
-  if (warp == 2 && lane == 0) {
-    bool ok = true;
-    int prev = 0;
-    for (int k = 0; k <= kE; ++k) {
-      const int v = args.offsets[k];
-      sched.offs[k] = v;
-      if (v < prev || (int64_t)v > args.rows_alloc) ok = false;
-      prev = v;
-    }
-    if (sched.offs[0] < 0) ok = false;
-    int acc = 0;
-    for (int k = 0; k < kE; ++k) {
-      const int n = ok ? sched.offs[k + 1] - sched.offs[k] : 0;
-      sched.mt[k] = (n + BM - 1) / BM;
-      sched.prefix[k] = acc;
-      acc += sched.mt[k] * args.n_tiles;
-    }
-    sched.prefix[kE] = acc;
-    if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
-  }
+  if (warp == 2 && lane == 0) build_schedule(sched, args, BM);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;

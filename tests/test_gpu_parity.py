@@ -29,6 +29,7 @@ SMALL = {
     "bf16_down_n128": (W["mid_bf16"], dict(T=300, d=384, f=256, capacity_factor=2.0)),
     "bf16_no_drop": (W["mid_bf16"], dict(T=513, d=512, f=640, capacity_factor=4.0)),
     "bf16_skew_drop": (W["grok_skew"], dict(T=1024, d=256, f=512)),
+    "bf16_pair_ragged": (W["mid_bf16"], dict(T=1500, d=512, f=768)),
     "mid_bf16": (W["mid_bf16"], {}),
 }
 
