@@ -18,7 +18,9 @@
 // Schedule: persistent, one CTA per SM.  The tile list is every
 // (expert, 128-row block, N block); tiles of one expert are ordered N-block
 // major so CTAs running at the same time share weight tiles and row blocks in
-// L2.  Rows of an expert's last block that belong to the next expert are
+// L2 (row-block-major order measured 50% slower), and both operands are
+// loaded with an evict-last L2 policy (1-2% faster than the default policy;
+// evict-first on the weights was 13% slower).  Rows of an expert's last block that belong to the next expert are
 // computed but not stored.  Warp roles (192 threads):
 //   warp 0 lane 0 : TMA producer over a kStages ring (full/empty mbarriers)
 //   warp 1 lane 0 : MMA issuer; warp 1 owns the 512 TMEM columns
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ producer
       uint32_t it = 0;
       bool ok = true;
+      const uint64_t keep = policy_evict_last();
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         const Tile t = decode_tile(sched, L, C::BN_OUT);
         for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
@@ -193,17 +196,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
           uint8_t* b = sB + s * C::B_BYTES;
-          tma_load_2d(sA + s * A_BYTES, &tmA, &full[s], kb * BK, t.m0);
+          tma_load_2d_hint(sA + s * A_BYTES, &tmA, &full[s], kb * BK, t.m0, keep);
           if (MODE == kGateUp) {
 #pragma unroll
             for (int c = 0; c < C::kChunks / 2; ++c) {
-              tma_load_3d(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e);
-              tma_load_3d(b + (C::kChunks / 2 + c) * CHUNK_BYTES, &tmB1, &full[s], t.n0 + 64 * c, kb * BK, t.e);
+              tma_load_3d_hint(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e, keep);
+              tma_load_3d_hint(b + (C::kChunks / 2 + c) * CHUNK_BYTES, &tmB1, &full[s], t.n0 + 64 * c, kb * BK, t.e, keep);
             }
           } else {
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e);
+              tma_load_3d_hint(b + c * CHUNK_BYTES, &tmB0, &full[s], t.n0 + 64 * c, kb * BK, t.e, keep);
           }
         }
       }
