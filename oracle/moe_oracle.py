@@ -220,6 +220,127 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, capacity_factor, logit_bias
 
 
 # ----------------------------------------------------------------------------
+# 8-bit expert weights ("weights in the official release were quantized":
+# "Benchmarking xAI's Grok-1", section "Grok-1: In Practice"; "8-Bit
+# Quantization" in the feature list of "Let Grok spill the beans on Grok";
+# the n4n.ai page's "Tradeoffs" section on quantising the weights to cut
+# their memory).  The pages name no scheme; the reading taken is symmetric
+# int8 per output channel, weights only (activations stay in the layer dtype).
+# ----------------------------------------------------------------------------
+def quantize_int8(w):
+    """Per-output-channel symmetric int8 of weights stored [..., K, N] (channel = N).
+
+    An encoding, so every decision is stated in fp32 (IEEE, round to nearest even):
+      amax[n]  = max_k |w[k, n]|          (exact: w is bf16 or fp32)
+      scale[n] = amax[n] / 127            (fp32 division)
+      q[k, n]  = clamp(rint(w[k, n] / scale[n]), -127, 127)   (fp32 division)
+    A column of zeros gets scale 0 and codes 0.  Returns (q int8, scale float32).
+    """
+    a = np.asarray(w)
+    if a.dtype == np.uint16:
+        wf = np.zeros(a.shape, dtype=np.uint32)
+        wf.view(np.uint16)[..., 1::2] = a
+        wf = wf.view(np.float32)
+    else:
+        wf = a.astype(np.float32)
+    amax = np.max(np.abs(wf), axis=-2)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    r = (wf / safe[..., None, :]).astype(np.float32)
+    q = np.clip(np.rint(r), -127, 127)
+    q = np.where(scale[..., None, :] > 0, q, 0).astype(np.int8)
+    return q, scale
+
+
+def dequantize_int8(q, scale):
+    """w'[k, n] = q[k, n] * scale[n], in float64 (exact)."""
+    return np.asarray(q, dtype=np.float64) * np.asarray(scale, dtype=np.float64)[..., None, :]
+
+
+ROW_CODE_MAX = 32512  # 127 * 256: a row code splits into two int8 halves
+
+
+def quantize_rows(v):
+    """15-bit symmetric code of each activation row, decisions in IEEE fp32:
+      scale[r] = max_k |v[r, k]| / 32512                    (fp32 division)
+      code[r, k] = clamp(rint(v[r, k] / scale[r]), -32512, 32512)
+      hi = floor((code + 128) / 256),  lo = code - 256 * hi  (both in [-128, 127])
+    so that code = 256 * hi + lo exactly.  A row of zeros gets scale 0.
+    Input values are taken as fp32 (bf16 bit patterns are widened exactly).
+    Returns (hi int8, lo int8, scale float32)."""
+    a = np.asarray(v)
+    if a.dtype == np.uint16:
+        vf = np.zeros(a.shape, dtype=np.uint32)
+        vf.view(np.uint16)[..., 1::2] = a
+        vf = vf.view(np.float32)
+    else:
+        vf = a.astype(np.float32)
+    amax = np.max(np.abs(vf), axis=-1)
+    scale = (amax / np.float32(ROW_CODE_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    code = np.clip(np.rint((vf / safe[..., None]).astype(np.float32)), -ROW_CODE_MAX, ROW_CODE_MAX)
+    code = np.where(scale[..., None] > 0, code, 0).astype(np.int64)
+    hi = np.floor_divide(code + 128, 256)
+    lo = code - 256 * hi
+    return hi.astype(np.int8), lo.astype(np.int8), scale
+
+
+def dequantize_rows(hi, lo, scale):
+    """v'[r, k] = (256 * hi + lo) * scale[r], in float64 (exact)."""
+    code = 256 * np.asarray(hi, dtype=np.int64) + np.asarray(lo, dtype=np.int64)
+    return code.astype(np.float64) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+def layer_forward_w8(x, w_router, q_gate, s_gate, q_up, s_up, q_down, s_down, capacity_factor, logit_bias=None,
+                     top_k: int = 2, tokens=None):
+    """The layer with int8 expert weights, as the 8-bit path defines it.
+
+    Routing, capacity and combine are those of layer_forward.  Each expert sees
+    its rows through quantize_rows (x rows, then the fp32-rounded H rows), and
+    its weights as q * scale; every product is then exact, so the expert output
+    is computed exactly (in float64) from those codes:
+      g = rows(x) @ (q_gate * s_gate),  u = rows(x) @ (q_up * s_up)
+      H = silu(g) * u,   y = rows(fp32(H)) @ (q_down * s_down)
+    """
+    x = np.asarray(x)
+    T = x.shape[0]
+    E = np.asarray(w_router).shape[0]
+    lg = router_logits(x, w_router, logit_bias)
+    idx, w = top2_softmax(lg, top_k)
+    cap = capacity(T, top_k, E, capacity_factor)
+    disp = dispatch(idx, w, E, cap)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    out = np.zeros((tok.size, x.shape[1]), dtype=np.float64)
+    for e in range(E):
+        rows = [(i, j) for i, t in enumerate(tok) for j in range(top_k)
+                if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
+        if not rows:
+            continue
+        xr = dequantize_rows(*quantize_rows(x[[tok[i] for i, _ in rows]]))
+        h = silu(xr @ dequantize_int8(q_gate[e], s_gate[e])) * (xr @ dequantize_int8(q_up[e], s_up[e]))
+        hr = dequantize_rows(*quantize_rows(h.astype(np.float32)))
+        y = hr @ dequantize_int8(q_down[e], s_down[e])
+        for r, (i, j) in enumerate(rows):
+            out[i] += w[tok[i], j] * y[r]
+    res = dict(disp)
+    res.update({"logits": lg, "idx": idx, "w": w, "cap": cap, "tokens": tok, "out": out})
+    return res
+
+
+class DequantizedExperts:
+    """Expert weights given as (q [E, K, N] int8, scale [E, N]); indexing an expert
+    returns its dequantized float64 matrix, so layer_forward can run on them
+    without materialising every expert at once."""
+
+    def __init__(self, q, scale):
+        self.q, self.scale = q, scale
+        self.shape = q.shape
+
+    def __getitem__(self, e):
+        return dequantize_int8(self.q[e], self.scale[e])
+
+
+# ----------------------------------------------------------------------------
 # statistics the pages define
 # ----------------------------------------------------------------------------
 def expert_batch_size(global_batch: int, seq_len: int, num_experts: int = 8, top_k: int = 2) -> float:

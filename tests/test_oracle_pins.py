@@ -253,10 +253,116 @@ def pin_bf16_decoding(o):
     np.testing.assert_array_equal(o.to_f64(bits), [1.0, -2.0, 0.25, 0.0, -0.0, 3.140625])
 
 
+def pin_quantize_int8(o):
+    rng = np.random.default_rng(12)
+    w = (rng.standard_normal((3, 40, 24)) * rng.random((1, 1, 24)) * 4).astype(np.float32)
+    w[1, :, 5] = 0.0  # an all-zero output channel
+    q, sc = o.quantize_int8(w)
+    assert q.dtype == np.int8 and sc.dtype == np.float32 and sc.shape == (3, 24)
+    # scale is the channel's max magnitude over 127 (channel = last axis)
+    np.testing.assert_array_equal(sc, (np.abs(w).max(axis=1) / np.float32(127)).astype(np.float32))
+    assert sc[1, 5] == 0 and np.all(q[1, :, 5] == 0)
+    # the largest magnitude of every non-zero channel maps to +-127
+    am = np.abs(w).argmax(axis=1)
+    for e in range(3):
+        for n in range(24):
+            if sc[e, n] > 0:
+                assert abs(int(q[e, am[e, n], n])) == 127
+    assert np.abs(q.astype(int)).max() <= 127
+    # nearest code: round-trip error at most half a step (+ fp32 division slack)
+    err = np.abs(o.dequantize_int8(q, sc) - w)
+    assert np.all(err <= sc[:, None, :] * (0.5 + 1e-6))
+    # symmetric
+    qn, _ = o.quantize_int8(-w)
+    np.testing.assert_array_equal(qn, -q)
+    # weights that are exactly k * 2^-4 with max |k| = 127 quantize to k
+    k = rng.integers(-127, 128, size=(2, 16, 8)).astype(np.float32)
+    k[:, 0, :] = 127
+    qk, sk = o.quantize_int8(k * np.float32(0.0625))
+    np.testing.assert_array_equal(qk, k.astype(np.int8))
+    # bf16 bit patterns are accepted and mean the same values
+    bits = (w.view(np.uint32) >> 16).astype(np.uint16)
+    wb = (bits.astype(np.uint32) << 16).view(np.float32)
+    qb, sb = o.quantize_int8(bits)
+    qf, sf = o.quantize_int8(wb)
+    np.testing.assert_array_equal(qb, qf)
+    np.testing.assert_array_equal(sb, sf)
+
+
+def pin_quantized_layer_uses_dequantized_weights(o):
+    rng = np.random.default_rng(13)
+    T, d, f = 7, 5, 6
+    x, wr, wg, wu, wd = rand_layer(rng, T, d, f, 8)
+    qs = [o.quantize_int8(m) for m in (wg, wu, wd)]
+    deq = [o.dequantize_int8(q, s) for q, s in qs]
+    lazy = [o.DequantizedExperts(q, s) for q, s in qs]
+    a = o.layer_forward(x, wr, *deq, 2.0)["out"]
+    b = o.layer_forward(x, wr, *lazy, 2.0)["out"]
+    np.testing.assert_array_equal(a, b)
+    lg, pairs, ref = bf_layer(x.tolist(), wr.tolist(), deq[0].tolist(), deq[1].tolist(), deq[2].tolist(),
+                              o.capacity(T, 2, 8, 2.0))
+    np.testing.assert_allclose(a, ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_quantize_rows(o):
+    rng = np.random.default_rng(14)
+    v = (rng.standard_normal((6, 300)) * np.array([[1e-3], [1.0], [50.0], [0.0], [3.0], [7.0]])).astype(np.float32)
+    hi, lo, sc = o.quantize_rows(v)
+    assert hi.dtype == np.int8 and lo.dtype == np.int8 and sc.dtype == np.float32
+    code = 256 * hi.astype(int) + lo.astype(int)
+    assert np.abs(code).max() <= 32512 and lo.min() >= -128 and lo.max() <= 127
+    np.testing.assert_array_equal(sc, (np.abs(v).max(axis=1) / np.float32(32512)).astype(np.float32))
+    assert sc[3] == 0 and np.all(code[3] == 0)
+    # the largest magnitude of each non-zero row codes to +-32512
+    am = np.abs(v).argmax(axis=1)
+    for r in range(6):
+        if sc[r] > 0:
+            assert abs(code[r, am[r]]) == 32512
+    # nearest code: half a step (+ fp32 division slack)
+    err = np.abs(o.dequantize_rows(hi, lo, sc) - v)
+    assert np.all(err <= sc[:, None] * (0.5 + 1e-6))
+    # hi/lo split: hi = floor((code + 128) / 256) for a few hand values
+    for c, h, l in [(0, 0, 0), (127, 0, 127), (128, 1, -128), (-128, 0, -128), (-129, -1, 127),
+                    (32512, 127, 0), (-32512, -127, 0), (383, 1, 127), (384, 2, -128)]:
+        hh, ll = np.floor_divide(c + 128, 256), c - 256 * np.floor_divide(c + 128, 256)
+        assert (hh, ll) == (h, l)
+    vv = np.array([[1.0, -1.0, 0.5, 127.0 / 256]], dtype=np.float32) * np.float32(32512 / 256)
+    h2, l2, s2 = o.quantize_rows(vv)
+    assert s2[0] == np.float32(2.0 ** -8)  # 127 / 32512, exact
+    np.testing.assert_array_equal(256 * h2.astype(int) + l2.astype(int), [[32512, -32512, 16256, 127 * 127]])
+
+
+def pin_int8_layer_exact(o):
+    # the 8-bit layer equals the float layer run on the dequantised weights and rows
+    rng = np.random.default_rng(15)
+    T, d, f = 9, 6, 5
+    x, wr, wg, wu, wd = rand_layer(rng, T, d, f, 8)
+    q = [o.quantize_int8(m) for m in (wg, wu, wd)]
+    r = o.layer_forward_w8(x, wr, q[0][0], q[0][1], q[1][0], q[1][1], q[2][0], q[2][1], 2.0)
+    deq = [o.dequantize_int8(*qq) for qq in q]
+    lg = o.router_logits(x, wr)
+    idx, w = o.top2_softmax(lg)
+    disp = o.dispatch(idx, w, 8, o.capacity(T, 2, 8, 2.0))
+    ref = np.zeros((T, d))
+    for t in range(T):
+        for j in range(2):
+            if disp["slot_of"][t, j] < 0:
+                continue
+            e = idx[t, j]
+            xr = o.dequantize_rows(*o.quantize_rows(x[t:t + 1]))[0]
+            g = [sum(xr[k] * deq[0][e][k, n] for k in range(d)) for n in range(f)]
+            u = [sum(xr[k] * deq[1][e][k, n] for k in range(d)) for n in range(f)]
+            h = np.array([gi / (1 + math.exp(-gi)) * ui for gi, ui in zip(g, u)])
+            hr = o.dequantize_rows(*o.quantize_rows(h.astype(np.float32)[None, :]))[0]
+            ref[t] += w[t, j] * np.array([sum(hr[k] * deq[2][e][k, n] for k in range(f)) for n in range(d)])
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [pin_router_logits, pin_top2_brute_force, pin_softmax_closed_form, pin_zero_router,
             pin_scale_invariance, pin_capacity_values, pin_dispatch_brute_force, pin_no_drop,
             pin_hand_built_drop, pin_layer_dense_brute_force, pin_identity_experts,
-            pin_two_expert_dense, pin_bf16_decoding]
+            pin_two_expert_dense, pin_bf16_decoding, pin_quantize_int8,
+            pin_quantized_layer_uses_dequantized_weights, pin_quantize_rows, pin_int8_layer_exact]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -343,7 +449,62 @@ MUTANTS = {
     "capacity_off_by_one": dict(dispatch=_dispatch_off_by_one),
     "capacity_floor": dict(capacity=lambda T, k, E, cf: T if math.isinf(cf) else int(math.floor(cf * T * k / E))),
     "gate_up_swapped": dict(swiglu_hidden=lambda x, g, u: _orig_hidden(x, u, g)),
+    "quant_per_row": dict(quantize_int8=lambda w: _quant_rows(w)),
+    "quant_scale_128": dict(quantize_int8=lambda w: _quant_div(w, 128.0)),
+    "quant_floor": dict(quantize_int8=lambda w: _quant_floor(w)),
+    "rows_hi_rounds": dict(quantize_rows=lambda v: _rows_round_hi(v)),
+    "rows_no_h_requant": dict(layer_forward_w8=lambda *a, **k: _w8_skip_h(*a, **k)),
 }
+
+
+def _rows_round_hi(v):
+    hi, lo, s = _orig_rows(v)
+    code = 256 * hi.astype(np.int64) + lo
+    h2 = np.rint(code / 256.0).astype(np.int64)
+    return np.clip(h2, -128, 127).astype(np.int8), (code - 256 * h2).clip(-128, 127).astype(np.int8), s
+
+
+def _w8_skip_h(x, wr, qg, sg, qu, su, qd, sd, cf, logit_bias=None, top_k=2, tokens=None):
+    saved = O.quantize_rows
+    calls = {"n": 0}
+
+    def only_first(v):
+        calls["n"] += 1
+        if calls["n"] % 2 == 0:  # pass H through unquantised
+            v = np.asarray(v, dtype=np.float64)
+            return np.zeros(v.shape, np.int8), np.zeros(v.shape, np.int8), np.zeros(v.shape[:-1], np.float32)
+        return saved(v)
+    O.quantize_rows = only_first
+    try:
+        return _orig_w8(x, wr, qg, sg, qu, su, qd, sd, cf, logit_bias, top_k, tokens)
+    finally:
+        O.quantize_rows = saved
+
+
+_orig_rows = O.quantize_rows
+_orig_w8 = O.layer_forward_w8
+
+
+def _quant_rows(w):
+    q, s = _orig_quant(np.swapaxes(np.asarray(w, dtype=np.float32), -1, -2))
+    return np.swapaxes(q, -1, -2), s
+
+
+def _quant_div(w, m):
+    wf = np.asarray(w, dtype=np.float32)
+    s = (np.abs(wf).max(axis=-2) / np.float32(m)).astype(np.float32)
+    q = np.clip(np.rint(wf / np.where(s > 0, s, 1)[..., None, :]), -127, 127).astype(np.int8)
+    return q, s
+
+
+def _quant_floor(w):
+    wf = np.asarray(w, dtype=np.float32)
+    s = (np.abs(wf).max(axis=-2) / np.float32(127)).astype(np.float32)
+    q = np.clip(np.floor(wf / np.where(s > 0, s, 1)[..., None, :]), -127, 127).astype(np.int8)
+    return q, s
+
+
+_orig_quant = O.quantize_int8
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -353,6 +514,6 @@ def test_planted_mistake_is_caught(name):
     for pin in ALL_PINS:
         try:
             pin(m)
-        except AssertionError:
+        except Exception:  # a failed assertion, or a pin that cannot even run on the mutant
             failures += 1
     assert failures >= 1, f"no pin catches mutant {name}"
