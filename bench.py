@@ -238,6 +238,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--shape", default=None, help="T,d,f override of the workload (profiling cases)")
+    ap.add_argument("--int8", action="store_true", help="int8 expert weights (weight-only, per-channel scales)")
     args = ap.parse_args()
     w = configs.WORKLOADS[args.workload]
     if args.shape:
@@ -300,7 +301,11 @@ def main():
             "x_perm": torch.empty((rows, w.d), dtype=tdt, device=dev)}
     stream = torch.cuda.current_stream(dev)
     names = ["router", "dispatch", "gate_up", "down", "combine"]
-    launches_per_step = 8  # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1
+    qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"]) if args.int8 else None
+    ws8 = (torch.empty((max(moe.lib.moe_expert_ffn_w8_workspace_size(cfg.ref), 16),), dtype=torch.uint8, device=dev)
+           if args.int8 else None)
+    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes)
+    launches_per_step = 10 if args.int8 else 8
 
     def step(ev=None):
         if ev:
@@ -311,10 +316,15 @@ def main():
         moe.dispatch(cfg, x, buf["idx"], buf["w"], out=disp, ws=buf["ws"])
         if ev:
             ev[2].record(stream)
-        moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
+        if qw is not None:
+            # int8 experts: gate/up and down in one call (both timed under "gate_up")
+            moe.expert_ffn_w8(cfg, disp["x_perm"], disp["offsets"], qw, disp["row_scale"], y=buf["y"], ws=ws8)
+        else:
+            moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
         if ev:
             ev[3].record(stream)
-        moe.expert_down(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], y=buf["y"])
+        if qw is None:
+            moe.expert_down(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], y=buf["y"])
         if ev:
             ev[4].record(stream)
         moe.combine(cfg, buf["y"], disp["slot_of"], buf["w"], weights_applied=True, out=buf["out"])
@@ -380,7 +390,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.storage == "bf16" else "f32",
             "data": "synthetic (seeded Philox4x32-10 normal inputs, random-init weights)",
-            "config": workload_config(w), "tflops": tflops,
+            "config": dict(workload_config(w), expert_weights="int8" if args.int8 else w.storage), "tflops": tflops,
             "tensor_frac_layer": tflops / peak,
             "kernels_ms": per_kernel, "counts_kept": counts_kept, "n_kept": n_kept,
             "gpu_launches": launches_per_step * args.steps, "roofline": roofline, "clocks": clk}
@@ -458,10 +468,30 @@ def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
     n_used = int(used.sum().item())
     weight_bytes = n_used * 3 * w.d * w.f * 2
     gbs = weight_bytes / (ms / 1000.0) / 1e9
-    return {"workload": w.name, "calls": w.calls, "ms_per_call": ms / w.calls,
-            "tokens_per_s": w.T * w.calls / (ms / 1000.0), "expert_weight_gb_per_call": weight_bytes / w.calls / 1e9,
-            "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
-            "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm"}
+    res = {"workload": w.name, "calls": w.calls, "ms_per_call": ms / w.calls,
+           "tokens_per_s": w.T * w.calls / (ms / 1000.0), "expert_weight_gb_per_call": weight_bytes / w.calls / 1e9,
+           "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+           "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm",
+           "kernel": "decode_gemm_kernel (weights on the MMA M side)"}
+    # the same calls with int8 expert weights (per-channel scales, int8 tensor cores)
+    qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"])
+    ws8 = torch.empty(moe.lib.moe_workspace_size_w8(cfg.ref), dtype=torch.uint8, device=dev)
+    for i in range(3):
+        moe.layer_forward_w8(cfg, xs[i], W["wr"], qw, out=out, ws=ws8)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for i in range(w.calls):
+        moe.layer_forward_w8(cfg, xs[i], W["wr"], qw, out=out, ws=ws8)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms8 = a.elapsed_time(b)
+    bytes8 = n_used * (3 * w.d * w.f + w.f * 2 * 4 + w.d * 4)  # int8 codes + fp32 scales of the used experts
+    gbs8 = bytes8 / (ms8 / 1000.0) / 1e9
+    res["int8_weights"] = {"ms_per_call": ms8 / w.calls, "tokens_per_s": w.T * w.calls / (ms8 / 1000.0),
+                           "expert_weight_gb_per_call": bytes8 / w.calls / 1e9, "achieved_gbs": gbs8,
+                           "frac": gbs8 / peaks["hbm_gbs"], "speedup_vs_bf16": ms / ms8}
+    del qw, ws8
+    return res
 
 
 if __name__ == "__main__":

@@ -197,6 +197,53 @@ MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void*
                                     const void* w_down, void* out_host, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
 
+/* 8-bit expert weights ("Benchmarking xAI's Grok-1", section "Grok-1: In
+ * Practice": the released weights were quantised; "Let Grok spill the beans
+ * on Grok": 8-bit quantisation; the pages give no scheme).  Weight-only,
+ * symmetric, one scale per output channel, every decision in IEEE fp32:
+ *   scale[e, n] = max_k |w[e, k, n]| / 127
+ *   q[e, k, n]  = clamp(rint(w[e, k, n] / scale[e, n]), -127, 127)  (0 if scale = 0)
+ * w: bf16 [E, K, N] (cfg->dtype must be MOE_BF16); q: int8 [E, K, N];
+ * scale: fp32 [E, N].  N must be a multiple of 64.  Gate and up are [E, d, f]
+ * (channel = f), down is [E, f, d] (channel = d). */
+MOE_API moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q,
+                                       float* scale, moe_stream_t stream);
+
+/* moe_expert_ffn with int8 expert weights, on the int8 tensor cores.
+ * Every weight is q * scale (per output channel, from moe_quantize_int8);
+ * every activation row entering a GEMM (rows of x_perm, then rows of H) is
+ * held as a 15-bit code with a per-row scale (finer than bf16):
+ *   s_r = max_k |v_k| / 32512,  c_k = clamp(rint(v_k / s_r), -32512, 32512)
+ * split exactly as c = 256 * hi + lo into two int8 planes, so every MMA is an
+ * exact int8 x int8 -> int32 product and the expert output is
+ *   s_w[n] * s_r * (256 * acc_hi + acc_lo)   (fp32).
+ * H is formed in fp32 and re-coded the same way before the down projection.
+ * Built for the weight-streaming regime (few tokens per expert; the weights
+ * are the MMA's M operand and tokens its N operand, 32 per tile).
+ * ws: moe_expert_ffn_w8_workspace_size bytes, laid out (256-byte aligned) as
+ * x codes hi [T*2, d] int8 | lo [T*2, d] int8 | scale [T*2] fp32 | H [T*2, f]
+ * fp32 | H codes hi [T*2, f] | lo [T*2, f] | scale [T*2] | up to four K-split
+ * partial outputs [4, T*2, d] fp32 (summed in a fixed order into y);
+ * y [T*2, d] fp32.  d must be a multiple of 256 (the down pass covers 256
+ * output channels per tile). */
+MOE_API size_t moe_expert_ffn_w8_workspace_size(const moe_config_t* cfg);
+MOE_API moe_status_t moe_expert_ffn_w8(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                                       const int8_t* q_gate, const float* s_gate, const int8_t* q_up,
+                                       const float* s_up, const int8_t* q_down, const float* s_down,
+                                       const float* row_scale, float* y, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/* Workspace of moe_layer_forward_w8: moe_workspace_size plus the scratch of
+ * moe_expert_ffn_w8. */
+MOE_API size_t moe_workspace_size_w8(const moe_config_t* cfg);
+
+/* moe_layer_forward with int8 expert weights (router weight stays bf16). */
+MOE_API moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const void* w_router,
+                                          const float* logit_bias, const int8_t* q_gate, const float* s_gate,
+                                          const int8_t* q_up, const float* s_up, const int8_t* q_down,
+                                          const float* s_down, void* out, int32_t* stats, void* ws,
+                                          size_t ws_bytes, moe_stream_t stream);
+
 /* Largest T accepted by moe_dispatch_noalloc. */
 #define MOE_NOALLOC_MAX_TOKENS (1 << 20)
 

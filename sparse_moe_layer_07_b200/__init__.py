@@ -7,7 +7,7 @@ points without the ``moe_`` prefix; they only check and marshal arguments
 PyTorch when the caller does not pass them.  Every step of the layer runs in
 the library's CUDA kernels: there is no fallback of any kind, and importing
 this package fails if the library has not been built
-(``python -m sparse_moe_layer_07_b200.build``).
+(``python sparse_moe_layer_07_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -21,7 +21,8 @@ __all__ = [
     "MoEError", "Config", "LIB_PATH", "lib", "abi_version", "capacity", "workspace_size",
     "dispatch_workspace_size", "router_topk", "dispatch", "expert_ffn", "expert_gate_up",
     "expert_down", "combine", "layer_forward", "layer_forward_host", "get_device_error",
-    "STATUS", "DEVERR", "dispatch_noalloc", "NOALLOC_MAX_TOKENS",
+    "STATUS", "DEVERR", "dispatch_noalloc", "NOALLOC_MAX_TOKENS", "quantize_int8", "expert_ffn_w8",
+    "layer_forward_w8", "QuantizedExperts", "w8_workspace_views",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -47,9 +48,12 @@ class _CConfig(ctypes.Structure):
                 ("reserved", ctypes.c_int32)]
 
 
+_BUILD_HINT = "build it with `python sparse_moe_layer_07_b200/build.py`"
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_moe_layer_07_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: {_BUILD_HINT}")
     L = ctypes.CDLL(LIB_PATH)
     P = ctypes.c_void_p
     cfgp = ctypes.POINTER(_CConfig)
@@ -71,9 +75,17 @@ def _load():
         "moe_layer_forward_host": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32], ctypes.c_int),
         "moe_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+        "moe_quantize_int8": ([cfgp, P, ctypes.c_int64, ctypes.c_int64, P, P, P], ctypes.c_int),
+        "moe_expert_ffn_w8_workspace_size": ([cfgp], sz),
+        "moe_workspace_size_w8": ([cfgp], sz),
+        "moe_expert_ffn_w8": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_layer_forward_w8": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
-        fn = getattr(L, name)
+        try:
+            fn = getattr(L, name)
+        except AttributeError as exc:
+            raise ImportError(f"{LIB_PATH} lacks {name} (out of date): {_BUILD_HINT}") from exc
         fn.argtypes = args
         fn.restype = res
     return L
@@ -280,6 +292,75 @@ def layer_forward_host(cfg: Config, x_host, w_router, w_gate, w_up, w_down, out_
                                       _dev_ptr(ws), ws.numel(), _stream(stream, w_router.device)),
            "moe_layer_forward_host")
     return out_host
+
+
+def quantize_int8(cfg: Config, w, q=None, scale=None, stream=None):
+    """Per-output-channel int8 codes and fp32 scales of expert weights w [E, K, N] (bf16)."""
+    E, K, N = w.shape
+    if q is None:
+        q = torch.empty((E, K, N), dtype=torch.int8, device=w.device)
+    if scale is None:
+        scale = torch.empty((E, N), dtype=torch.float32, device=w.device)
+    _check(lib.moe_quantize_int8(cfg.ref, _dev_ptr(w), K, N, _dev_ptr(q), _dev_ptr(scale), _stream(stream, w.device)),
+           "moe_quantize_int8")
+    return q, scale
+
+
+class QuantizedExperts:
+    """int8 expert weights of one layer: codes and per-channel scales of gate, up and down."""
+
+    def __init__(self, cfg: Config, w_gate, w_up, w_down, stream=None):
+        self.q_gate, self.s_gate = quantize_int8(cfg, w_gate, stream=stream)
+        self.q_up, self.s_up = quantize_int8(cfg, w_up, stream=stream)
+        self.q_down, self.s_down = quantize_int8(cfg, w_down, stream=stream)
+
+    def ptrs(self):
+        return [_dev_ptr(t) for t in (self.q_gate, self.s_gate, self.q_up, self.s_up, self.q_down, self.s_down)]
+
+
+def _round256(n):
+    return (n + 255) // 256 * 256
+
+
+def w8_workspace_views(cfg: Config, ws):
+    """Named views into the scratch of expert_ffn_w8 (layout stated in include/moe.h)."""
+    rows, d, f = cfg.T * cfg.top_k, cfg.d, cfg.f
+    spec = [("x_hi", rows * d, torch.int8, (rows, d)), ("x_lo", rows * d, torch.int8, (rows, d)),
+            ("x_scale", rows * 4, torch.float32, (rows,)), ("h", rows * f * 4, torch.float32, (rows, f)),
+            ("h_hi", rows * f, torch.int8, (rows, f)), ("h_lo", rows * f, torch.int8, (rows, f)),
+            ("h_scale", rows * 4, torch.float32, (rows,)),
+            ("y_parts", 4 * rows * d * 4, torch.float32, (4, rows, d))]
+    views, o = {}, 0
+    for name, nbytes, dt, shape in spec:
+        views[name] = ws[o:o + nbytes].view(dt).view(shape)
+        o += _round256(nbytes)
+    return views
+
+
+def expert_ffn_w8(cfg: Config, x_perm, offsets, qw: QuantizedExperts, row_scale=None, y=None, ws=None,
+                  stream=None):
+    """SwiGLU experts with int8 weights over the grouped rows.  Returns (y, ws)."""
+    if y is None:
+        y = _empty((cfg.T * cfg.top_k, cfg.d), torch.float32, x_perm)
+    if ws is None:
+        ws = _empty((max(lib.moe_expert_ffn_w8_workspace_size(cfg.ref), 1),), torch.uint8, x_perm)
+    _check(lib.moe_expert_ffn_w8(cfg.ref, _dev_ptr(x_perm), _dev_ptr(offsets), *qw.ptrs(), _dev_ptr(row_scale),
+                                 _dev_ptr(y), _dev_ptr(ws), ws.numel(), _stream(stream, x_perm.device)),
+           "moe_expert_ffn_w8")
+    return y, ws
+
+
+def layer_forward_w8(cfg: Config, x, w_router, qw: QuantizedExperts, logit_bias=None, out=None, stats=None, ws=None,
+                     stream=None):
+    """The whole layer with int8 expert weights; returns out [T, d]."""
+    if out is None:
+        out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
+    if ws is None:
+        ws = _empty((max(lib.moe_workspace_size_w8(cfg.ref), 1),), torch.uint8, x)
+    _check(lib.moe_layer_forward_w8(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(logit_bias), *qw.ptrs(),
+                                    _dev_ptr(out), _dev_ptr(stats), _dev_ptr(ws), ws.numel(),
+                                    _stream(stream, x.device)), "moe_layer_forward_w8")
+    return out
 
 
 def get_device_error(clear: bool = True) -> int:

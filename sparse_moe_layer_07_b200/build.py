@@ -1,6 +1,7 @@
 """Build libmoe_b200.so (all CUDA sources, sm_100a) next to this file.
 
-Usage: python -m sparse_moe_layer_07_b200.build [--force]
+Usage: python sparse_moe_layer_07_b200/build.py [--force] [-v]
+(run it by path: importing the package loads the library it builds)
 Objects go to <repo>/_build/; the shared library is written in-tree so it
 travels with the source tree.  Only nvcc and the CUDA headers are needed (no
 GPU): the driver entry points are resolved at run time.

@@ -61,8 +61,42 @@ moe_status_t validate_config(const moe_config_t* cfg);
 // Device facts of the current device (cached per device).
 moe_status_t current_ctx(Ctx& out);
 
-// Encodes a tiled TMA descriptor (driver entry point resolved once).
+// Encodes a tiled TMA descriptor (driver entry point resolved once); bf16 elements.
 bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz);
+bool encode_tmap_dtype(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+                       CUtensorMapDataType dtype);
+
+// Per-output-channel int8 quantisation of E matrices [K, N] (bf16 in).
+cudaError_t launch_quantize_int8(int E, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
+                                 cudaStream_t s);
+
+// Expert GEMMs with the weights on the MMA's M side (small token counts,
+// bf16 weights).
+cudaError_t launch_decode_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
+                                  const void* wg, const void* wu, void* h, cudaStream_t s, const Ctx& ctx);
+cudaError_t launch_decode_down(const moe_config_t& c, const void* h, const int32_t* offsets,
+                               const void* wd, const float* row_scale, float* y, cudaStream_t s,
+                               const Ctx& ctx);
+
+// 15-bit row codes (hi/lo int8 planes + per-row scale) of the first offsets[E]
+// rows of src ([rows, K], bf16 or fp32).
+cudaError_t launch_quantize_rows(const void* src, bool src_f32, const int32_t* offsets, int64_t max_rows,
+                                 int64_t K, int8_t* hi, int8_t* lo, float* scale, int num_sms, cudaStream_t s);
+
+// Expert GEMMs on the int8 tensor cores: int8 weights x row-code planes.
+cudaError_t launch_i8_gate_up(const moe_config_t& c, const int8_t* x_hi, const int8_t* x_lo,
+                              const float* x_scale, const int32_t* offsets, const int8_t* qg,
+                              const float* sg, const int8_t* qu, const float* su, float* h, cudaStream_t s,
+                              const Ctx& ctx);
+// K splits of the int8 down pass (1, 2 or 4).
+int down_splits(const moe_config_t& c);
+// Writes down_splits(c) K-split partials [splits, T*k, d] fp32; launch_sum_partials adds them into y.
+cudaError_t launch_i8_down(const moe_config_t& c, const int8_t* h_hi, const int8_t* h_lo, const float* h_scale,
+                           const int32_t* offsets, const int8_t* qd, const float* sd, const float* row_scale,
+                           float* y_parts, cudaStream_t s, const Ctx& ctx);
+cudaError_t launch_sum_partials(const moe_config_t& c, const float* y_parts, const int32_t* offsets, float* y,
+                                cudaStream_t s, const Ctx& ctx);
 
 }  // namespace moe

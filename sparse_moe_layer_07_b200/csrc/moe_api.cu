@@ -122,8 +122,15 @@ Layout layout_of(const moe_config_t& c) {
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Batches averaging at most 64 rows per expert stream the expert weights
+// rather than reuse them; they run on the kernel that puts the weights on
+// the MMA's M side and spends no tensor time on padded token rows.
+bool weight_streaming(const moe_config_t& c) { return c.T * (int64_t)c.top_k <= 64 * (int64_t)c.E; }
+
 moe_status_t run_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets, const void* wg,
                          const void* wu, void* h, cudaStream_t s, const Ctx& ctx) {
+  if (c.dtype == MOE_BF16 && weight_streaming(c))
+    return cuda_status(launch_decode_gate_up(c, x_perm, offsets, wg, wu, h, s, ctx));
   if (c.dtype == MOE_BF16) return cuda_status(launch_tc_gate_up(c, x_perm, offsets, wg, wu, h, s, ctx));
   return cuda_status(launch_ffn_simt_gate_up(c, static_cast<const float*>(x_perm), offsets,
                                              static_cast<const float*>(wg), static_cast<const float*>(wu),
@@ -132,6 +139,8 @@ moe_status_t run_gate_up(const moe_config_t& c, const void* x_perm, const int32_
 
 moe_status_t run_down(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
                       const float* row_scale, float* y, cudaStream_t s, const Ctx& ctx) {
+  if (c.dtype == MOE_BF16 && weight_streaming(c))
+    return cuda_status(launch_decode_down(c, h, offsets, wd, row_scale, y, s, ctx));
   if (c.dtype == MOE_BF16) return cuda_status(launch_tc_down(c, h, offsets, wd, row_scale, y, s, ctx));
   return cuda_status(launch_ffn_simt_down(c, static_cast<const float*>(h), offsets, static_cast<const float*>(wd),
                                           row_scale, y, s, ctx));
@@ -145,6 +154,12 @@ moe_status_t current_ctx(Ctx& out) { return get_ctx(out); }
 
 bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                  const uint32_t* box, CUtensorMapSwizzle swz) {
+  return encode_tmap_dtype(map, base, rank, dims, strides_bytes, box, swz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+bool encode_tmap_dtype(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+                       CUtensorMapDataType dtype) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -155,7 +170,7 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -363,6 +378,147 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
   if (cudaMemcpyAsync(out_host, w8 + L.out, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(cudaStreamSynchronize(stream));
+}
+
+moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
+                               moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (K <= 0 || N <= 0 || K > ((int64_t)1 << 20) || N > ((int64_t)1 << 20)) return MOE_ERR_INVALID_ARG;
+  if (N % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!w || !q || !scale || !aligned16(w) || !aligned16(q) || !aligned16(scale)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_int8(cfg->E, w, K, N, q, scale, stream));
+}
+
+static moe_status_t check_w8(const moe_config_t* cfg, const void* qg, const float* sg, const void* qu,
+                             const float* su, const void* qd, const float* sd) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16 || cfg->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!qg || !sg || !qu || !su || !qd || !sd) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(qg) || !aligned16(qu) || !aligned16(qd) || !aligned16(sg) || !aligned16(su) || !aligned16(sd))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// Scratch of the int8-weight expert FFN, carved in this order:
+// row codes of x_perm (hi, lo planes and per-row scales), H in fp32, row codes of H.
+struct W8Layout {
+  size_t x_hi, x_lo, x_scale, h, h_hi, h_lo, h_scale, y_parts, total;
+};
+
+W8Layout w8_layout_of(const moe_config_t& c) {
+  W8Layout L;
+  const size_t rows = (size_t)slot_rows(c);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += round_up(bytes);
+    return at;
+  };
+  L.x_hi = take(rows * c.d);
+  L.x_lo = take(rows * c.d);
+  L.x_scale = take(rows * 4);
+  L.h = take(rows * c.f * 4);
+  L.h_hi = take(rows * c.f);
+  L.h_lo = take(rows * c.f);
+  L.h_scale = take(rows * 4);
+  L.y_parts = take(4 * rows * c.d * 4);
+  L.total = o;
+  return L;
+}
+
+cudaError_t run_ffn_w8(const moe_config_t& c, const void* x_perm, const int32_t* offsets, const int8_t* qg,
+                       const float* sg, const int8_t* qu, const float* su, const int8_t* qd, const float* sd,
+                       const float* row_scale, float* y, uint8_t* ws, cudaStream_t s, const Ctx& ctx) {
+  const W8Layout L = w8_layout_of(c);
+  const int64_t rows = slot_rows(c);
+  int8_t* x_hi = reinterpret_cast<int8_t*>(ws + L.x_hi);
+  int8_t* x_lo = reinterpret_cast<int8_t*>(ws + L.x_lo);
+  float* x_sc = reinterpret_cast<float*>(ws + L.x_scale);
+  float* h = reinterpret_cast<float*>(ws + L.h);
+  int8_t* h_hi = reinterpret_cast<int8_t*>(ws + L.h_hi);
+  int8_t* h_lo = reinterpret_cast<int8_t*>(ws + L.h_lo);
+  float* h_sc = reinterpret_cast<float*>(ws + L.h_scale);
+  cudaError_t e = launch_quantize_rows(x_perm, false, offsets, rows, c.d, x_hi, x_lo, x_sc, ctx.num_sms, s);
+  if (e == cudaSuccess) e = launch_i8_gate_up(c, x_hi, x_lo, x_sc, offsets, qg, sg, qu, su, h, s, ctx);
+  if (e == cudaSuccess) e = launch_quantize_rows(h, true, offsets, rows, c.f, h_hi, h_lo, h_sc, ctx.num_sms, s);
+  float* y_parts = reinterpret_cast<float*>(ws + L.y_parts);
+  if (e == cudaSuccess) e = launch_i8_down(c, h_hi, h_lo, h_sc, offsets, qd, sd, row_scale, y_parts, s, ctx);
+  if (e == cudaSuccess) e = launch_sum_partials(c, y_parts, offsets, y, s, ctx);
+  return e;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_expert_ffn_w8_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return w8_layout_of(*cfg).total;
+}
+
+size_t moe_workspace_size_w8(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg).total + w8_layout_of(*cfg).total;
+}
+
+moe_status_t moe_expert_ffn_w8(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                               const int8_t* q_gate, const float* s_gate, const int8_t* q_up, const float* s_up,
+                               const int8_t* q_down, const float* s_down, const float* row_scale, float* y, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_w8(cfg, q_gate, s_gate, q_up, s_up, q_down, s_down);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !offsets || !y || !aligned16(x_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < w8_layout_of(*cfg).total) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return cuda_status(run_ffn_w8(*cfg, x_perm, offsets, q_gate, s_gate, q_up, s_up, q_down, s_down, row_scale, y,
+                                static_cast<uint8_t*>(ws), stream, ctx));
+}
+
+moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const void* w_router,
+                                  const float* logit_bias, const int8_t* q_gate, const float* s_gate,
+                                  const int8_t* q_up, const float* s_up, const int8_t* q_down, const float* s_down,
+                                  void* out, int32_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_w8(cfg, q_gate, s_gate, q_up, s_up, q_down, s_down);
+  if (st != MOE_OK) return st;
+  if (!w_router || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias))) return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) return MOE_OK;
+  if (!ws || ws_bytes < moe_workspace_size_w8(cfg) || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (!x || !out || !aligned16(x) || !aligned16(out) || (stats && !aligned16(stats))) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  const Layout L = layout_of(c);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(w8 + L.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(w8 + L.topk_w);
+  int32_t* route = reinterpret_cast<int32_t*>(w8 + L.route);
+  int32_t* offsets = route + 2 * c.E;
+  int32_t* perm = reinterpret_cast<int32_t*>(w8 + L.perm);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(w8 + L.slot_of);
+  float* row_scale = reinterpret_cast<float*>(w8 + L.row_scale);
+  void* x_perm = w8 + L.x_perm;
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  cudaError_t e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, route, route + c.E, offsets, perm, slot_of, row_scale,
+                        reinterpret_cast<int32_t*>(w8 + L.disp), stats, stream, ctx);
+  if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, x_perm, stream, ctx);
+  if (e == cudaSuccess)
+    e = run_ffn_w8(c, x_perm, offsets, q_gate, s_gate, q_up, s_up, q_down, s_down, row_scale, y, w8 + L.total, stream,
+                   ctx);
+  if (e == cudaSuccess) e = launch_combine(c, y, slot_of, topk_w, 1, out, stream, ctx);
+  return cuda_status(e);
 }
 
 moe_status_t moe_get_device_error(int32_t* code, int32_t clear) {

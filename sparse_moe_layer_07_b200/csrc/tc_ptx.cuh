@@ -134,6 +134,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem], int8 x int8 -> int32 (exact), one CTA.
+__device__ __forceinline__ void umma_s8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -180,6 +191,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
   return (1u << 4)                                  // D format: f32
          | (1u << 7)                                // A format: bf16
          | (1u << 10)                               // B format: bf16
+         | ((a_mn_major ? 1u : 0u) << 15)           // A major
+         | ((b_mn_major ? 1u : 0u) << 16)           // B major
+         | ((uint32_t)(N >> 3) << 17)               // N / 8
+         | ((uint32_t)(M >> 4) << 24);              // M / 16
+}
+
+// Instruction descriptor, kind::i8 with signed int8 A/B and int32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (2u << 4)                                  // D format: s32
+         | (1u << 7)                                // A format: signed int8
+         | (1u << 10)                               // B format: signed int8
          | ((a_mn_major ? 1u : 0u) << 15)           // A major
          | ((b_mn_major ? 1u : 0u) << 16)           // B major
          | ((uint32_t)(N >> 3) << 17)               // N / 8

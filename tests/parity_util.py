@@ -72,6 +72,21 @@ def run_steps(L: LayerInputs, keep_h=True):
     return r
 
 
+def run_steps_w8(L, qw):
+    """Router -> dispatch -> int8 expert FFN -> combine through the separate entry points."""
+    c, D = L.cfg, L.dev
+    idx, wts, logits = moe.router_topk(c, D["x"], D["wr"], D["bias"], want_logits=True)
+    disp = moe.dispatch(c, D["x"], idx, wts)
+    y, ws = moe.expert_ffn_w8(c, disp["x_perm"], disp["offsets"], qw, disp["row_scale"])
+    out = moe.combine(c, y, disp["slot_of"], wts, weights_applied=True)
+    torch.cuda.synchronize()
+    g = {"idx": idx.cpu().numpy(), "w": wts.cpu().numpy(), "logits": logits.cpu().numpy().astype(np.float64),
+         "out": out, "y": y, "ws": moe.w8_workspace_views(c, ws), "x_perm": disp["x_perm"]}
+    for k in ("counts_raw", "counts_kept", "offsets", "perm", "slot_of", "row_scale"):
+        g[k] = disp[k].cpu().numpy()
+    return g
+
+
 def logit_bound(x, wr, logits64, d):
     ax = np.abs(oracle.to_f64(x))
     aw = np.abs(oracle.to_f64(wr))

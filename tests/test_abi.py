@@ -13,9 +13,9 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 @pytest.fixture(scope="module")
 def moe():
-    from sparse_moe_layer_07_b200 import build
+    import __graft_entry__
 
-    build.build()
+    __graft_entry__.build()
     import sparse_moe_layer_07_b200 as m
 
     return m

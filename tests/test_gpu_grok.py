@@ -16,7 +16,8 @@ import torch
 import oracle
 from synth import configs
 
-from parity_util import LayerInputs, check_dispatch, check_layer_out, check_routing, run_steps, to_dev
+from parity_util import (LayerInputs, check_dispatch, check_layer_out, check_routing, run_steps, run_steps_w8,
+                         to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -106,3 +107,42 @@ def test_grok_decode_full_size(grok):
         res.append(check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"][i * w.T:(i + 1) * w.T], rows))
     REPORT["grok_decode"] = {"calls_checked": list(calls), "max_err_over_rms": [list(r) for r in res],
                              "experts_used": [int((g["counts_kept"] > 0).sum()) for _, g in outs]}
+
+
+def test_grok_decode_int8_full_size(grok):
+    """int8 expert weights at full Grok size: every code and scale against the
+    oracle's own quantisation, then the decode layer against the oracle's 8-bit
+    layer (its own codes for weights and rows)."""
+    import sparse_moe_layer_07_b200 as moe
+
+    host, dev = grok
+    w = W["grok_decode"]
+    cfg = moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16")
+    qw = moe.QuantizedExperts(cfg, dev["wg"], dev["wu"], dev["wd"])
+    torch.cuda.synchronize()
+    ref_q = {}
+    for name, gq, gs in (("wg", qw.q_gate, qw.s_gate), ("wu", qw.q_up, qw.s_up), ("wd", qw.q_down, qw.s_down)):
+        qs, ss = [], []
+        for e in range(8):
+            q, s = oracle.quantize_int8(host[name][e])
+            assert np.array_equal(gq[e].cpu().numpy(), q), (name, e)
+            assert np.array_equal(gs[e].cpu().numpy(), s), (name, e)
+            qs.append(q)
+            ss.append(s)
+        ref_q[name] = (np.stack(qs), np.stack(ss))
+    calls = (0, 99)
+    outs = []
+    for c in calls:
+        L = LayerInputs(w, call=c, host=host, dev_weights=dev)
+        g = run_steps_w8(L, qw)
+        assert int(g["offsets"][-1]) == 2 * w.T
+        check_routing(L, g, oracle.router_logits(L.x, L.wr))
+        check_dispatch(L, g)
+        outs.append((L, g))
+    # no capacity drop: tokens are independent, so one oracle call covers both batches
+    x_all = np.concatenate([L.x for L, _ in outs])
+    ref = oracle.layer_forward_w8(x_all, host["wr"], *ref_q["wg"], *ref_q["wu"], *ref_q["wd"], float("inf"))
+    res = [check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"][i * w.T:(i + 1) * w.T], np.arange(w.T))
+           for i, (L, g) in enumerate(outs)]
+    REPORT["grok_decode_int8"] = {"calls_checked": list(calls), "weight_codes_bit_exact": True,
+                                  "max_err_over_rms": [list(r) for r in res]}

@@ -30,6 +30,9 @@ SMALL = {
     "bf16_no_drop": (W["mid_bf16"], dict(T=513, d=512, f=640, capacity_factor=4.0)),
     "bf16_skew_drop": (W["grok_skew"], dict(T=1024, d=256, f=512)),
     "bf16_pair_ragged": (W["mid_bf16"], dict(T=1500, d=512, f=768)),
+    # at most 64 rows per expert on average: the weight-streaming (swap-AB) kernel
+    "bf16_stream_no_drop": (W["mid_bf16"], dict(T=96, d=256, f=384, capacity_factor=4.0)),
+    "bf16_stream_ragged": (W["mid_bf16"], dict(T=250, d=384, f=512)),
     "mid_bf16": (W["mid_bf16"], {}),
 }
 
