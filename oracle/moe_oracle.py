@@ -1,4 +1,4 @@
-"""Plain, slow, fp64 CPU oracle of the Grok-1-style sparse MoE layer forward pass.
+"""Plain, slow, fp64 CPU oracle of the Grok-1-style sparse MoE layer (forward and backward).
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports or calls this
 module: only the tests, the smoke check and the benchmark's CPU-baseline leg
@@ -216,6 +216,91 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, capacity_factor, logit_bias
     res.update({"logits": lg, "idx": idx, "w": w, "cap": cap, "tokens": tok, "out": out})
     if keep_hidden:
         res["hidden"] = hidden
+    return res
+
+
+# ----------------------------------------------------------------------------
+# Backward pass (training).  The pages give only the forward pass; the
+# capacity drop is described as a training-time rule ([Routing], capacity
+# paragraph), so training differentiates this same forward.  Reading: the
+# gradient of L = sum(out * dout) with respect to x, W_r, the logit bias and
+# the expert weights, with the discrete steps (the top-2 choice and the
+# capacity mask) held fixed: they are piecewise constant, so their derivative
+# is zero wherever it exists.  The gradient reaches the router only through
+# the softmax weights of the two selected logits.
+# ----------------------------------------------------------------------------
+def silu_grad(z: np.ndarray) -> np.ndarray:
+    """d/dz [z * sigmoid(z)] = sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, logit_bias=None, top_k: int = 2):
+    """Gradients of sum(out * dout) for the layer of layer_forward.
+
+    Per kept assignment (t, j) with expert e and weight w = w[t, j]:
+      g = x_t W_gate[e], u = x_t W_up[e], h = silu(g) * u, y = h W_down[e]
+      out_t += w * y                                   ([Arch], [EP])
+    so, with dy = w * dout_t:
+      dweight[t, j] = <dout_t, y>
+      dW_down[e] += h^T dy,   dh = dy W_down[e]^T
+      dg = dh * u * silu'(g), du = dh * silu(g)
+      dW_gate[e] += x_t^T dg, dW_up[e] += x_t^T du,  dx_t += dg W_gate[e]^T + du W_up[e]^T
+    Dropped assignments contribute nothing (dweight = 0).  The softmax over the
+    selected logits w_j = exp(l_j) / sum_i exp(l_i) gives
+      dlogits[t, idx[t, j]] = w_j * (dweight_j - sum_i w_i * dweight_i)
+    and the router logits l = x W_r^T + bias give
+      dW_r = dlogits^T x,  dx += dlogits W_r,  dbias = sum_t dlogits[t].
+    Returns the forward intermediates of layer_forward plus dx [T, d],
+    dw_router [E, d], dbias [E], dw_gate [E, d, f], dw_up [E, d, f],
+    dw_down [E, f, d], dlogits [T, E] and dweight [T, k], all float64.
+    """
+    x64 = to_f64(x)
+    T, d = x64.shape
+    wr = to_f64(w_router)
+    E = wr.shape[0]
+    g_dout = to_f64(dout)
+    lg = router_logits(x, w_router, logit_bias)
+    idx, w = top2_softmax(lg, top_k)
+    cap = capacity(T, top_k, E, capacity_factor)
+    disp = dispatch(idx, w, E, cap)
+    f = np.asarray(w_gate[0]).shape[1]
+    dx = np.zeros((T, d))
+    dwg = np.zeros((E, d, f))
+    dwu = np.zeros((E, d, f))
+    dwd = np.zeros((E, f, d))
+    dweight = np.zeros((T, top_k))
+    for e in range(E):
+        pairs = [(t, j) for t in range(T) for j in range(top_k) if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
+        if not pairs:
+            continue
+        ts = np.array([t for t, _ in pairs])
+        js = np.array([j for _, j in pairs])
+        wg, wu, wd = to_f64(w_gate[e]), to_f64(w_up[e]), to_f64(w_down[e])
+        xr = x64[ts]
+        g = xr @ wg
+        u = xr @ wu
+        h = silu(g) * u
+        y = h @ wd
+        dy = w[ts, js][:, None] * g_dout[ts]
+        dweight[ts, js] = np.sum(g_dout[ts] * y, axis=1)
+        dwd[e] = h.T @ dy
+        dh = dy @ wd.T
+        dg = dh * u * silu_grad(g)
+        du = dh * silu(g)
+        dwg[e] = xr.T @ dg
+        dwu[e] = xr.T @ du
+        np.add.at(dx, ts, dg @ wg.T + du @ wu.T)
+    dlogits = np.zeros((T, E))
+    mean = np.sum(w * dweight, axis=1)
+    for t in range(T):
+        for j in range(top_k):
+            dlogits[t, idx[t, j]] += w[t, j] * (dweight[t, j] - mean[t])
+    dx += dlogits @ wr
+    res = dict(disp)
+    res.update({"logits": lg, "idx": idx, "w": w, "cap": cap, "dx": dx, "dw_router": dlogits.T @ x64,
+                "dbias": dlogits.sum(axis=0), "dw_gate": dwg, "dw_up": dwu, "dw_down": dwd, "dlogits": dlogits,
+                "dweight": dweight})
     return res
 
 

@@ -358,11 +358,97 @@ def pin_int8_layer_exact(o):
     np.testing.assert_allclose(r["out"], ref, rtol=1e-12, atol=1e-12)
 
 
+# ----------------------------------------------------------------------------
+# backward pass
+# ----------------------------------------------------------------------------
+def _bwd_case(seed, T=6, d=5, f=4, E=8, bias=True):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d))
+    b = rng.standard_normal(E) * 0.5 if bias else None
+    wg = rng.standard_normal((E, d, f)) * 0.7
+    wu = rng.standard_normal((E, d, f)) * 0.7
+    wd = rng.standard_normal((E, f, d)) * 0.7
+    go = rng.standard_normal((T, d))
+    return x, wr, b, wg, wu, wd, go
+
+
+def pin_backward_finite_differences(o):
+    # every gradient entry against central differences of L = sum(out * dout), on a case
+    # with dropped assignments (cap = 2 for 6 tokens x 2 slots over 8 experts) and a bias
+    x, wr, b, wg, wu, wd, go = _bwd_case(21)
+    cf = 1.0
+    r = o.layer_backward(x, wr, wg, wu, wd, cf, go, logit_bias=b)
+    assert r["dropped"] > 0
+    assert o.near_tie_gap(r["logits"]).min() > 1e-3
+
+    def loss(x_, wr_, b_, wg_, wu_, wd_):
+        return float(np.sum(o.layer_forward(x_, wr_, wg_, wu_, wd_, cf, logit_bias=b_)["out"] * go))
+
+    args = [x, wr, b, wg, wu, wd]
+    names = ["dx", "dw_router", "dbias", "dw_gate", "dw_up", "dw_down"]
+    eps = 1e-6
+    for a_i, name in enumerate(names):
+        base = args[a_i]
+        num = np.zeros(base.shape)
+        for pos in np.ndindex(base.shape):
+            hi = [a.copy() if i == a_i else a for i, a in enumerate(args)]
+            lo = [a.copy() if i == a_i else a for i, a in enumerate(args)]
+            hi[a_i][pos] += eps
+            lo[a_i][pos] -= eps
+            num[pos] = (loss(*hi) - loss(*lo)) / (2 * eps)
+        np.testing.assert_allclose(r[name], num, rtol=1e-6, atol=1e-6, err_msg=name)
+
+
+def pin_backward_autograd(o):
+    # a larger case against torch autograd (float64) of the forward restated with the
+    # oracle's routing decisions held fixed
+    import torch
+
+    T, d, f, E = 40, 12, 10, 8
+    x, wr, b, wg, wu, wd, go = _bwd_case(22, T, d, f, E)
+    cf = 1.25
+    r = o.layer_backward(x, wr, wg, wu, wd, cf, go, logit_bias=b)
+    assert r["dropped"] > 0
+    tx, twr, tb, twg, twu, twd = (torch.tensor(a, requires_grad=True) for a in (x, wr, b, wg, wu, wd))
+    lg = tx @ twr.T + tb
+    idx = torch.tensor(r["idx"], dtype=torch.int64)
+    sel = torch.gather(lg, 1, idx)
+    wsm = torch.softmax(sel, dim=1)
+    out = torch.zeros(T, d, dtype=torch.float64)
+    for t in range(T):
+        for j in range(2):
+            if r["slot_of"][t, j] < 0:
+                continue
+            e = int(idx[t, j])
+            hdn = torch.nn.functional.silu(tx[t] @ twg[e]) * (tx[t] @ twu[e])
+            out = out.index_add(0, torch.tensor([t]), (wsm[t, j] * (hdn @ twd[e]))[None])
+    (out * torch.tensor(go)).sum().backward()
+    for name, ten in zip(["dx", "dw_router", "dbias", "dw_gate", "dw_up", "dw_down"], (tx, twr, tb, twg, twu, twd)):
+        np.testing.assert_allclose(r[name], ten.grad.numpy(), rtol=1e-10, atol=1e-10, err_msg=name)
+
+
+def pin_backward_dropped_token(o):
+    # a token whose two assignments are both dropped has out = 0 whatever its x is, so
+    # its dx, dlogits and dweight are 0; gradients are linear in dout
+    x, wr, b, wg, wu, wd, go = _bwd_case(23, T=8)
+    bias = np.array([40.0, 30.0, 0, 0, 0, 0, 0, 0])
+    r = o.layer_backward(x, wr, wg, wu, wd, 0.5, go, logit_bias=bias)
+    cap = o.capacity(8, 2, 8, 0.5)
+    assert cap == 1 and (r["idx"] == [0, 1]).all()
+    assert np.all(r["dx"][1:] == 0) and np.all(r["dlogits"][1:] == 0) and np.all(r["dweight"][1:] == 0)
+    assert np.any(r["dx"][0] != 0)
+    r2 = o.layer_backward(x, wr, wg, wu, wd, 0.5, 3.0 * go, logit_bias=bias)
+    for k in ("dx", "dw_router", "dw_gate", "dw_up", "dw_down"):
+        np.testing.assert_allclose(r2[k], 3.0 * r[k], rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [pin_router_logits, pin_top2_brute_force, pin_softmax_closed_form, pin_zero_router,
             pin_scale_invariance, pin_capacity_values, pin_dispatch_brute_force, pin_no_drop,
             pin_hand_built_drop, pin_layer_dense_brute_force, pin_identity_experts,
             pin_two_expert_dense, pin_bf16_decoding, pin_quantize_int8,
-            pin_quantized_layer_uses_dequantized_weights, pin_quantize_rows, pin_int8_layer_exact]
+            pin_quantized_layer_uses_dequantized_weights, pin_quantize_rows, pin_int8_layer_exact,
+            pin_backward_finite_differences, pin_backward_autograd, pin_backward_dropped_token]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -408,6 +494,17 @@ def _mutant(**overrides):
             for k, v in saved.items():
                 setattr(O, k, v)
     m.layer_forward = layer_forward
+
+    def layer_backward(*a, **k):
+        saved = {kk: getattr(O, kk) for kk in overrides}
+        try:
+            for kk, v in overrides.items():
+                setattr(O, kk, v)
+            return overrides.get("layer_backward", saved.get("layer_backward", O.layer_backward))(*a, **k)
+        finally:
+            for kk, v in saved.items():
+                setattr(O, kk, v)
+    m.layer_backward = layer_backward
     return m
 
 
@@ -454,7 +551,40 @@ MUTANTS = {
     "quant_floor": dict(quantize_int8=lambda w: _quant_floor(w)),
     "rows_hi_rounds": dict(quantize_rows=lambda v: _rows_round_hi(v)),
     "rows_no_h_requant": dict(layer_forward_w8=lambda *a, **k: _w8_skip_h(*a, **k)),
+    "bwd_silu_grad_sigmoid_only": dict(silu_grad=lambda z: 1.0 / (1.0 + np.exp(-z))),
+    "bwd_no_router_term_in_dx": dict(layer_backward=lambda *a, **k: _bwd_no_router_dx(*a, **k)),
+    "bwd_softmax_grad_without_mean": dict(layer_backward=lambda *a, **k: _bwd_no_mean(*a, **k)),
+    "bwd_gate_up_grads_swapped": dict(layer_backward=lambda *a, **k: _bwd_swap_gu(*a, **k)),
 }
+
+
+def _bwd_no_router_dx(x, wr, *a, **k):
+    r = _orig_bwd(x, wr, *a, **k)
+    r["dx"] = r["dx"] - r["dlogits"] @ O.to_f64(wr)
+    return r
+
+
+def _bwd_no_mean(x, wr, *a, **k):
+    r = _orig_bwd(x, wr, *a, **k)
+    extra = np.zeros_like(r["dlogits"])
+    mean = np.sum(r["w"] * r["dweight"], axis=1)
+    for t in range(extra.shape[0]):
+        for j in range(r["idx"].shape[1]):
+            extra[t, r["idx"][t, j]] += r["w"][t, j] * mean[t]
+    r["dlogits"] = r["dlogits"] + extra
+    r["dx"] = r["dx"] + extra @ O.to_f64(wr)
+    r["dw_router"] = r["dlogits"].T @ O.to_f64(x)
+    r["dbias"] = r["dlogits"].sum(axis=0)
+    return r
+
+
+def _bwd_swap_gu(*a, **k):
+    r = _orig_bwd(*a, **k)
+    r["dw_gate"], r["dw_up"] = r["dw_up"], r["dw_gate"]
+    return r
+
+
+_orig_bwd = O.layer_backward
 
 
 def _rows_round_hi(v):
