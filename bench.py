@@ -239,6 +239,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--shape", default=None, help="T,d,f override of the workload (profiling cases)")
     ap.add_argument("--int8", action="store_true", help="int8 expert weights (weight-only, per-channel scales)")
+    ap.add_argument("--no-train", action="store_true", help="skip the training pair (forward + backward)")
+    ap.add_argument("--train-steps", type=int, default=5)
+    ap.add_argument("--unfused", action="store_true",
+                    help="separate down and combine kernels instead of the fused down-combine")
     args = ap.parse_args()
     w = configs.WORKLOADS[args.workload]
     if args.shape:
@@ -304,8 +308,15 @@ def main():
     qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"]) if args.int8 else None
     ws8 = (torch.empty((max(moe.lib.moe_expert_ffn_w8_workspace_size(cfg.ref), 16),), dtype=torch.uint8, device=dev)
            if args.int8 else None)
-    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes)
-    launches_per_step = 10 if args.int8 else 8
+    # the one-call layer's kernels: bf16 tensor-core batches sum the down outputs into token
+    # order (zero + down + rounding pass, no y buffer, no separate combine)
+    fused = (qw is None and not args.unfused and w.storage == "bf16" and w.T * 2 > 64 * w.E and w.d % 256 == 0)
+    if fused:
+        buf["dc_ws"] = torch.empty(moe.lib.moe_expert_down_combine_workspace_size(cfg.ref), dtype=torch.uint8,
+                                   device=dev)
+    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes);
+    # fused: router 1, dispatch 3 + gather 1, gate/up 1, zero + down + rounding 3 (9)
+    launches_per_step = 10 if args.int8 else (9 if fused else 8)
 
     def step(ev=None):
         if ev:
@@ -316,6 +327,16 @@ def main():
         moe.dispatch(cfg, x, buf["idx"], buf["w"], out=disp, ws=buf["ws"])
         if ev:
             ev[2].record(stream)
+        if fused:
+            moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
+            if ev:
+                ev[3].record(stream)
+            moe.expert_down_combine(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], disp["perm"],
+                                    out=buf["out"], ws=buf["dc_ws"])
+            if ev:
+                ev[4].record(stream)
+                ev[5].record(stream)
+            return
         if qw is not None:
             # int8 experts: gate/up and down in one call (both timed under "gate_up")
             moe.expert_ffn_w8(cfg, disp["x_perm"], disp["offsets"], qw, disp["row_scale"], y=buf["y"], ws=ws8)
@@ -377,7 +398,8 @@ def main():
     gu_ms = per_kernel["gate_up"]
     achieved = gu_flops / (gu_ms / 1000.0) / 1e12
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    roofline = {"bound": "tensor", "kernel": "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)",
+    gu_name = "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)"
+    roofline = {"bound": "tensor", "kernel": gu_name,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
                 "traffic": measured_traffic(w.name),
@@ -392,38 +414,69 @@ def main():
             "data": "synthetic (seeded Philox4x32-10 normal inputs, random-init weights)",
             "config": dict(workload_config(w), expert_weights="int8" if args.int8 else w.storage), "tflops": tflops,
             "tensor_frac_layer": tflops / peak,
-            "kernels_ms": per_kernel, "counts_kept": counts_kept, "n_kept": n_kept,
+            "kernels_ms": per_kernel,
+            "path": ("down-combine fused: down sums into token order (its time includes the zeroing and "
+                     "rounding passes; combine 0)") if fused else "separate down and combine",
+            "counts_kept": counts_kept, "n_kept": n_kept,
             "gpu_launches": launches_per_step * args.steps, "roofline": roofline, "clocks": clk}
 
-    # ---- end to end: host x in, host out, through the C entry point with host buffers
+    # ---- end to end: host x in, host out, through the C entry points with host buffers.
+    # Headline: moe_layer_forward_host_batches, one batch per step, every step's x copied
+    # in and its out copied back inside the timed region (overlapped with the compute of
+    # the neighbouring steps).  Also reported: the one-batch call, which waits per batch.
     if not args.no_e2e:
-        ws_full = torch.empty(moe.workspace_size(cfg), dtype=torch.uint8, device=dev)
+        ws_full = torch.empty(moe.workspace_size_host_batches(cfg), dtype=torch.uint8, device=dev)
         x_host = torch.from_numpy(np.ascontiguousarray(x_np))
         x_host = (x_host.view(torch.bfloat16) if w.storage == "bf16" else x_host).pin_memory()
-        out_host = torch.empty((w.T, w.d), dtype=tdt).pin_memory()
-        for _ in range(2):
-            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_host, ws_full,
-                                   logit_bias=bias_d)
+        out_ring = [torch.empty((w.T, w.d), dtype=tdt).pin_memory() for _ in range(2)]
+
+        def run_batches(n):
+            moe.layer_forward_host_batches(cfg, [x_host] * n, W["wr"], W["wg"], W["wu"], W["wd"],
+                                           [out_ring[i % 2] for i in range(n)], ws_full, logit_bias=bias_d,
+                                           stream=stream)
+
+        run_batches(args.warmup)
         if world > 1:
             dist.barrier()
+        torch.cuda.synchronize(dev)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.steps):
-            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_host, ws_full,
-                                   logit_bias=bias_d)
+        run_batches(args.steps)
         b.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(a.elapsed_time(b), dev, world)
         nbytes = w.T * w.d * (2 if w.storage == "bf16" else 4)
+        # the one-batch entry point (copy in, layer, copy out, wait) for comparison
+        single_steps = min(args.steps, 10)
+        moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
+                               logit_bias=bias_d, stream=stream)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(single_steps):
+            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
+                                   logit_bias=bias_d, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        single_ms = max_over_ranks(a.elapsed_time(b), dev, world) / single_steps
         line["e2e"] = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
                        "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms / args.steps,
-                       "api": "moe_layer_forward_host (pinned host x/out, device-resident weights)"}
+                       "api": "moe_layer_forward_host_batches (pinned host x/out, one batch per step, copies "
+                              "overlapped with the neighbouring steps' compute; device-resident weights)",
+                       "one_batch_call": {"ms_per_step": single_ms,
+                                          "value": tokens / args.steps / (single_ms / 1000.0),
+                                          "api": "moe_layer_forward_host (copy in, layer, copy out, wait)"}}
         del ws_full
 
     # ---- decode (weight streaming) on the same Grok-shape weights
     if not args.no_decode and w.name == "grok_prefill" and not args.shape:
         line["decode"] = decode_bench(moe, W, dev, stream, peaks, peak_src, world)
+
+    # ---- training step (forward that keeps its state + backward) on the same batch
+    if (not args.no_train and w.name == "grok_prefill" and w.storage == "bf16" and w.d % 256 == 0
+            and w.f % 256 == 0):
+        line["train"] = train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, args.train_steps)
 
     if rank == 0 and world == 1 and not args.no_cpu and host is not None:
         t, n = oracle_sample(w, host, x_np, args.cpu_tokens, 7)
@@ -435,6 +488,56 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, steps):
+    """Forward-for-training + backward of the layer; backward FLOPs = 12*d*f per kept row
+    (dH, dX over gate and up, and the three weight gradients) + 4*T*d*E for the router."""
+    import torch
+
+    from synth import normal
+
+    ws = torch.empty(moe.workspace_size_train(cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
+    dout = torch.from_numpy(normal(configs.SEED, 907, (cfg.T, cfg.d), dtype="bf16")).view(torch.bfloat16).to(dev)
+    E, d, f = cfg.E, cfg.d, cfg.f
+    grads = {"dx": torch.empty((cfg.T, d), dtype=torch.bfloat16, device=dev),
+             "dw_router": torch.empty((E, d), dtype=torch.float32, device=dev),
+             "dbias": torch.empty((E,), dtype=torch.float32, device=dev),
+             "dw_gate": torch.empty((E, d, f), dtype=torch.float32, device=dev),
+             "dw_up": torch.empty((E, d, f), dtype=torch.float32, device=dev),
+             "dw_down": torch.empty((E, f, d), dtype=torch.float32, device=dev)}
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        moe.layer_forward_train(cfg, x, W["wr"], W["wg"], W["wu"], W["wd"], ws, logit_bias=bias_d, out=out,
+                                stream=stream)
+        if ev:
+            ev[1].record(stream)
+        moe.layer_backward(cfg, x, W["wr"], W["wg"], W["wu"], W["wd"], dout, ws, grads=grads, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    fwd = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs) / steps, dev, world)
+    bwd = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evs) / steps, dev, world)
+    bwd_flops = 12.0 * n_kept * d * f + 4.0 * cfg.T * d * E
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tf = bwd_flops / (bwd / 1000.0) / 1e12
+    res = {"steps": steps, "forward_train_ms": fwd, "backward_ms": bwd,
+           "tokens_per_s": world * cfg.T / ((fwd + bwd) / 1000.0),
+           "backward_tflops": tf, "backward_frac": tf / peak,
+           "backward_algorithmic": "12*d*f*N_kept + 4*T*d*E FLOP", "gpu_launches_per_step": 8 + 10,
+           "grad_dtype": "fp32 weight gradients, bf16 dx"}
+    del ws, grads
+    return res
 
 
 def decode_bench(moe, W, dev, stream, peaks, peak_src, world):

@@ -27,7 +27,8 @@
  *     or keeps a pointer after a call returns.
  *   - Tensors are dense row-major.  Buffers must be 16-byte aligned.
  *   - Work is enqueued on `stream` (a cudaStream_t); calls return before the
- *     GPU finishes, except moe_layer_forward_host and moe_get_device_error.
+ *     GPU finishes, except moe_layer_forward_host, moe_layer_forward_host_batches
+ *     and moe_get_device_error.
  *   - Argument errors are reported synchronously, before anything is launched:
  *     MOE_ERR_INVALID_ARG (null pointer, bad size, misalignment),
  *     MOE_ERR_UNSUPPORTED (E != 8, top_k != 2, d or f not a multiple of 128
@@ -168,6 +169,23 @@ MOE_API moe_status_t moe_expert_down(const moe_config_t* cfg, const void* h, con
                              const void* w_down, const float* row_scale, float* y, void* ws,
                              size_t ws_bytes, moe_stream_t stream);
 
+/* Down projection with the combine fused (bf16 only, the tensor-core kernels
+ * for batches above the weight-streaming size; d a multiple of 256):
+ *   out[t, :] = sum over kept slots r of token t of row_scale[r] * (h[r, :] @ w_down[e])
+ * in fp32, rounded once to cfg->dtype: moe_expert_down followed by moe_combine
+ * with weights_applied = 1, bit for bit, without the y buffer (the down
+ * epilogue adds each row into an fp32 sum by token; with two terms per token
+ * the sum does not depend on their order).  h, offsets from moe_dispatch /
+ * moe_expert_gate_up; perm, row_scale from moe_dispatch; out [T, d] in
+ * cfg->dtype; ws: device scratch of moe_expert_down_combine_workspace_size(cfg)
+ * bytes (the fp32 sums).  MOE_ERR_UNSUPPORTED outside that scope (fp32,
+ * d % 256 != 0, or T * top_k <= 64 * E, where the weight-streaming kernels
+ * run instead).  moe_layer_forward uses this path in its scope. */
+MOE_API size_t moe_expert_down_combine_workspace_size(const moe_config_t* cfg);
+MOE_API moe_status_t moe_expert_down_combine(const moe_config_t* cfg, const void* h, const int32_t* offsets,
+                                     const void* w_down, const float* row_scale, const int32_t* perm, void* out,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Weighted combine back to token order ("The high-level architecture",
  * _dispatch_and_combine; weighted sum of the active experts' outputs):
  *   out[t, :] = sum over j = 0, 1 with slot_of[t, j] >= 0 of
@@ -196,6 +214,58 @@ MOE_API moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void*
                                     const float* logit_bias, const void* w_gate, const void* w_up,
                                     const void* w_down, void* out_host, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
+
+/* Bytes of device workspace needed by moe_layer_forward_host_batches:
+ * moe_workspace_size plus a second x and out staging slot; 0 for an invalid
+ * config. */
+MOE_API size_t moe_workspace_size_host_batches(const moe_config_t* cfg);
+
+/* The layer over n_batches independent batches of cfg->T tokens held in host
+ * memory (one layer call per batch, as moe_layer_forward_host computes it),
+ * with the copies overlapped with the compute: while batch i computes on
+ * `stream`, batch i+1 is copied in and batch i-1 copied out on two streams of
+ * the library's own, through two staging slots in ws.  Every batch's result is
+ * bit-identical to moe_layer_forward on the same x.  The pages define one
+ * forward call ("The high-level architecture", forward); this entry point only
+ * schedules many of them, it adds no arithmetic.
+ * x_host[i]: host [T, d] in cfg->dtype; out_host[i]: host [T, d]; both arrays
+ * hold n_batches pointers; entries may repeat (a repeated out_host buffer ends
+ * with the last batch written to it).  Page-locked buffers are needed for the
+ * copies to overlap.  Weights, logit_bias and ws are device memory; ws holds
+ * moe_workspace_size_host_batches(cfg) bytes.  The work is ordered after the
+ * work already in `stream`; the call returns when every out_host[i] is filled.
+ * n_batches == 0 does nothing.  The two copy streams and their events are
+ * created and destroyed inside the call (no device memory is allocated). */
+MOE_API moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_batches,
+                                            const void* const* x_host, const void* w_router,
+                                            const float* logit_bias, const void* w_gate, const void* w_up,
+                                            const void* w_down, void* const* out_host, void* ws,
+                                            size_t ws_bytes, moe_stream_t stream);
+
+/* Training: the forward pass that keeps what the backward needs, and the
+ * backward pass.  The pages describe the forward only; the backward is the
+ * derivative of that forward with the routing decisions (top-2 choice and
+ * capacity mask) held fixed: the gradient reaches the router through the
+ * softmax over the two selected logits ("Routing: top-2 without auxiliary
+ * loss"), and the experts through "Expert implementation: SwiGLU at scale".
+ * For L = sum(out * dout):
+ *   dx [T, d] (cfg->dtype), dw_router [E, d], dbias [E] (or NULL),
+ *   dw_gate, dw_up [E, d, f], dw_down [E, f, d]: fp32, overwritten.
+ * bf16 only, d and f multiples of 256 (MOE_ERR_UNSUPPORTED otherwise).
+ * ws: moe_workspace_size_train(cfg) bytes; moe_layer_forward_train fills it
+ * (routing, grouped rows, H and the pre-activations G, U) and computes the
+ * same out as moe_layer_forward; moe_layer_backward reads it (same cfg, x and
+ * weights) and may be called again on it.  Every reduction has a fixed order:
+ * results do not depend on scheduling. */
+MOE_API size_t moe_workspace_size_train(const moe_config_t* cfg);
+MOE_API moe_status_t moe_layer_forward_train(const moe_config_t* cfg, const void* x, const void* w_router,
+                                     const float* logit_bias, const void* w_gate, const void* w_up,
+                                     const void* w_down, void* out, void* ws, size_t ws_bytes,
+                                     moe_stream_t stream);
+MOE_API moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const void* w_router,
+                                const void* w_gate, const void* w_up, const void* w_down, const void* dout,
+                                void* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up,
+                                float* dw_down, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* 8-bit expert weights ("Benchmarking xAI's Grok-1", section "Grok-1: In
  * Practice": the released weights were quantised; "Let Grok spill the beans

@@ -235,7 +235,8 @@ def silu_grad(z: np.ndarray) -> np.ndarray:
     return s * (1.0 + z * (1.0 - s))
 
 
-def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, logit_bias=None, top_k: int = 2):
+def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, logit_bias=None, top_k: int = 2,
+                   tokens=None):
     """Gradients of sum(out * dout) for the layer of layer_forward.
 
     Per kept assignment (t, j) with expert e and weight w = w[t, j]:
@@ -254,6 +255,10 @@ def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, log
     Returns the forward intermediates of layer_forward plus dx [T, d],
     dw_router [E, d], dbias [E], dw_gate [E, d, f], dw_up [E, d, f],
     dw_down [E, f, d], dlogits [T, E] and dweight [T, k], all float64.
+    With ``tokens`` (a subset), routing and capacity still run over all T, but
+    only the listed tokens' assignments are differentiated: their rows of dx,
+    dlogits and dweight are exact, the other rows are zero, and the parameter
+    gradients hold only those tokens' contributions.
     """
     x64 = to_f64(x)
     T, d = x64.shape
@@ -270,8 +275,9 @@ def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, log
     dwu = np.zeros((E, d, f))
     dwd = np.zeros((E, f, d))
     dweight = np.zeros((T, top_k))
+    tok = range(T) if tokens is None else sorted(set(int(t) for t in tokens))
     for e in range(E):
-        pairs = [(t, j) for t in range(T) for j in range(top_k) if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
+        pairs = [(t, j) for t in tok for j in range(top_k) if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
         if not pairs:
             continue
         ts = np.array([t for t, _ in pairs])
@@ -293,7 +299,7 @@ def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, log
         np.add.at(dx, ts, dg @ wg.T + du @ wu.T)
     dlogits = np.zeros((T, E))
     mean = np.sum(w * dweight, axis=1)
-    for t in range(T):
+    for t in tok:
         for j in range(top_k):
             dlogits[t, idx[t, j]] += w[t, j] * (dweight[t, j] - mean[t])
     dx += dlogits @ wr
@@ -302,6 +308,44 @@ def layer_backward(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, log
                 "dbias": dlogits.sum(axis=0), "dw_gate": dwg, "dw_up": dwu, "dw_down": dwd, "dlogits": dlogits,
                 "dweight": dweight})
     return res
+
+
+def expert_weight_grad_slices(x, w_router, w_gate, w_up, w_down, capacity_factor, dout, e, cols,
+                              logit_bias=None, top_k: int = 2):
+    """Slices of layer_backward's weight gradients for one expert, for layers too
+    large to differentiate whole: columns ``cols`` of dW_gate[e] and dW_up[e]
+    ([d, n]) and rows ``cols`` of dW_down[e] ([n, d]).  The same formulas
+    restricted to those hidden units: every hidden unit m of expert e only needs
+    g[:, m], u[:, m] and W_down[e][m, :], so
+      dW_down[e][m, :] = sum_r h[r, m] * dy[r, :]
+      dW_gate[e][:, m] = sum_r x_r * dg[r, m],  dW_up[e][:, m] = sum_r x_r * du[r, m]
+    over the kept rows r of expert e (routing and capacity over all tokens)."""
+    x64 = to_f64(x)
+    T = x64.shape[0]
+    E = np.asarray(w_router).shape[0]
+    lg = router_logits(x, w_router, logit_bias)
+    idx, w = top2_softmax(lg, top_k)
+    disp = dispatch(idx, w, E, capacity(T, top_k, E, capacity_factor))
+    pairs = [(t, j) for t in range(T) for j in range(top_k) if idx[t, j] == e and disp["slot_of"][t, j] >= 0]
+    cols = np.asarray(cols, dtype=np.int64)
+    d = x64.shape[1]
+    if not pairs:
+        return {"dw_gate_cols": np.zeros((d, cols.size)), "dw_up_cols": np.zeros((d, cols.size)),
+                "dw_down_rows": np.zeros((cols.size, d))}
+    ts = np.array([t for t, _ in pairs])
+    js = np.array([j for _, j in pairs])
+    xr = x64[ts]
+    wg = to_f64(np.asarray(w_gate[e])[:, cols])
+    wu = to_f64(np.asarray(w_up[e])[:, cols])
+    wd = to_f64(np.asarray(w_down[e])[cols, :])
+    g = xr @ wg
+    u = xr @ wu
+    h = silu(g) * u
+    dy = w[ts, js][:, None] * to_f64(dout)[ts]
+    dh = dy @ wd.T
+    dg = dh * u * silu_grad(g)
+    du = dh * silu(g)
+    return {"dw_gate_cols": xr.T @ dg, "dw_up_cols": xr.T @ du, "dw_down_rows": h.T @ dy}
 
 
 # ----------------------------------------------------------------------------

@@ -73,6 +73,13 @@ def _load():
         "moe_combine": ([cfgp, P, P, P, ctypes.c_int32, P, P], ctypes.c_int),
         "moe_layer_forward": ([cfgp, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_host": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_workspace_size_host_batches": ([cfgp], sz),
+        "moe_expert_down_combine_workspace_size": ([cfgp], sz),
+        "moe_workspace_size_train": ([cfgp], sz),
+        "moe_layer_forward_train": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_layer_backward": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_expert_down_combine": ([cfgp, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_layer_forward_host_batches": ([cfgp, ctypes.c_int64, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32], ctypes.c_int),
         "moe_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "moe_quantize_int8": ([cfgp, P, ctypes.c_int64, ctypes.c_int64, P, P, P], ctypes.c_int),
@@ -261,6 +268,18 @@ def expert_ffn(cfg: Config, x_perm, offsets, w_gate, w_up, w_down, row_scale=Non
     return h, y
 
 
+def expert_down_combine(cfg: Config, h, offsets, w_down, row_scale, perm, out=None, ws=None, stream=None):
+    """down x routing weight summed straight into token order (down + combine, no y)."""
+    if out is None:
+        out = _empty((cfg.T, cfg.d), cfg.torch_dtype, h)
+    if ws is None:
+        ws = _empty((max(lib.moe_expert_down_combine_workspace_size(cfg.ref), 1),), torch.uint8, h)
+    _check(lib.moe_expert_down_combine(cfg.ref, _dev_ptr(h), _dev_ptr(offsets), _dev_ptr(w_down), _dev_ptr(row_scale),
+                                       _dev_ptr(perm), _dev_ptr(out), _dev_ptr(ws), ws.numel(),
+                                       _stream(stream, h.device)), "moe_expert_down_combine")
+    return out
+
+
 def combine(cfg: Config, y, slot_of, topk_w=None, weights_applied: bool = True, out=None, stream=None):
     if out is None:
         out = _empty((cfg.T, cfg.d), cfg.torch_dtype, y)
@@ -292,6 +311,69 @@ def layer_forward_host(cfg: Config, x_host, w_router, w_gate, w_up, w_down, out_
                                       _dev_ptr(ws), ws.numel(), _stream(stream, w_router.device)),
            "moe_layer_forward_host")
     return out_host
+
+
+def workspace_size_host_batches(cfg: Config) -> int:
+    return lib.moe_workspace_size_host_batches(cfg.ref)
+
+
+def layer_forward_host_batches(cfg: Config, x_hosts, w_router, w_gate, w_up, w_down, out_hosts, ws, logit_bias=None,
+                               stream=None):
+    """The layer over several host-resident batches, copies overlapped with compute
+    (``moe_layer_forward_host_batches``); returns when every out_hosts[i] is filled."""
+    if len(x_hosts) != len(out_hosts):
+        raise ValueError("x_hosts and out_hosts must have the same length")
+    if any(t.is_cuda for t in list(x_hosts) + list(out_hosts)):
+        raise ValueError("x_hosts and out_hosts must be host tensors")
+    for t in list(x_hosts) + list(out_hosts):
+        if t.dtype != cfg.torch_dtype or t.numel() != cfg.T * cfg.d:
+            raise ValueError(f"host batches must be [T, d] = [{cfg.T}, {cfg.d}] of {cfg.dtype}")
+    n = len(x_hosts)
+    xs = (ctypes.c_void_p * max(n, 1))(*[_ptr(t) for t in x_hosts])
+    outs = (ctypes.c_void_p * max(n, 1))(*[_ptr(t) for t in out_hosts])
+    _check(lib.moe_layer_forward_host_batches(cfg.ref, n, ctypes.cast(xs, ctypes.c_void_p), _dev_ptr(w_router),
+                                              _dev_ptr(logit_bias), _dev_ptr(w_gate), _dev_ptr(w_up),
+                                              _dev_ptr(w_down), ctypes.cast(outs, ctypes.c_void_p), _dev_ptr(ws),
+                                              ws.numel(), _stream(stream, w_router.device)),
+           "moe_layer_forward_host_batches")
+    return out_hosts
+
+
+def workspace_size_train(cfg: Config) -> int:
+    return lib.moe_workspace_size_train(cfg.ref)
+
+
+def layer_forward_train(cfg: Config, x, w_router, w_gate, w_up, w_down, ws, logit_bias=None, out=None, stream=None):
+    """The layer forward that keeps the backward's inputs in ws (moe_workspace_size_train bytes)."""
+    if out is None:
+        out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
+    _check(lib.moe_layer_forward_train(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(logit_bias),
+                                       _dev_ptr(w_gate), _dev_ptr(w_up), _dev_ptr(w_down), _dev_ptr(out),
+                                       _dev_ptr(ws), ws.numel(), _stream(stream, x.device)), "moe_layer_forward_train")
+    return out
+
+
+def layer_backward(cfg: Config, x, w_router, w_gate, w_up, w_down, dout, ws, grads=None, want_dbias=True,
+                   stream=None):
+    """Gradients of sum(out * dout) after layer_forward_train on the same ws.  Returns a dict of
+    dx (layer dtype) and fp32 dw_router, dbias (or None), dw_gate, dw_up, dw_down."""
+    E, d, f = cfg.E, cfg.d, cfg.f
+    g = dict(grads or {})
+    g.setdefault("dx", _empty((cfg.T, d), cfg.torch_dtype, x))
+    g.setdefault("dw_router", _empty((E, d), torch.float32, x))
+    if want_dbias:
+        g.setdefault("dbias", _empty((E,), torch.float32, x))
+    else:
+        g["dbias"] = None
+    g.setdefault("dw_gate", _empty((E, d, f), torch.float32, x))
+    g.setdefault("dw_up", _empty((E, d, f), torch.float32, x))
+    g.setdefault("dw_down", _empty((E, f, d), torch.float32, x))
+    _check(lib.moe_layer_backward(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(w_gate), _dev_ptr(w_up),
+                                  _dev_ptr(w_down), _dev_ptr(dout), _dev_ptr(g["dx"]), _dev_ptr(g["dw_router"]),
+                                  _dev_ptr(g["dbias"]), _dev_ptr(g["dw_gate"]), _dev_ptr(g["dw_up"]),
+                                  _dev_ptr(g["dw_down"]), _dev_ptr(ws), ws.numel(), _stream(stream, x.device)),
+           "moe_layer_backward")
+    return g
 
 
 def quantize_int8(cfg: Config, w, q=None, scale=None, stream=None):

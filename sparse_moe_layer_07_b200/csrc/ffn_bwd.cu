@@ -1,0 +1,548 @@
+// Backward of the expert FFNs on the tcgen05 tensor cores (training).
+//
+// The pages give the forward pass only ("How does Grok-1 use a
+// mixture-of-experts design?", sections "Expert implementation: SwiGLU at
+// scale" and "Expert parallelism vs. tensor parallelism"); training
+// differentiates that forward with the routing decisions held fixed.  For
+// the kept rows r of expert e (token t = perm[r], weight w = row_scale[r]),
+// with G = X W_gate, U = X W_up, H = silu(G) * U saved by the forward:
+//   kDH : dHu[r, :] = dout[t, :] W_down[e]^T        (A = dout rows, B = W_down K-major)
+//         epilogue: dH = w * dHu,  dG = dH * U * silu'(G),  dU = dH * silu(G),
+//         and a per-tile partial of <dHu, H> (= the routing weight's gradient
+//         <dout, y>), summed later in a fixed order
+//   kDX : dx[t, :] += dG[r, :] W_gate[e]^T + dU[r, :] W_up[e]^T
+//         (K runs over both halves; B = W_gate / W_up read K-major straight from
+//         their [E, d, f] layout; the epilogue adds into an fp32 sum by token:
+//         two terms per token, so the order of the adds does not matter)
+//   kWG : dW[e] = A_e^T B_e over the rows of expert e  (A, B MN-major:
+//         dW_down = H^T (w * dout),  dW_gate = X^T dG,  dW_up = X^T dU); K is
+//         the ragged row count, the rows past the expert's end in its last K
+//         block are zeroed in shared memory before the MMA.
+// Pipeline as in ffn_tc.cu: persistent CTAs, warp 0 TMA, warp 1 MMA + TMEM
+// (two 128 x 256 fp32 accumulators), warps 2-5 epilogue; every wait bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+using namespace ptx;
+
+constexpr int kE = 8;
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kAccStride = 256;
+constexpr int CHUNK = 64 * BK * 2;      // 8 KB: 64 x 64 bf16
+constexpr int A_BYTES = 2 * CHUNK;      // 16 KB: 128 x 64
+constexpr int B_BYTES = 4 * CHUNK;      // 32 KB: 256 x 64
+constexpr int STAGE = A_BYTES + B_BYTES;
+constexpr int kStages = 4;
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE + 256;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+enum Mode { kDH = 0, kDX = 1, kWG = 2 };
+
+struct BwdArgs {
+  const int32_t* offsets;  // [E + 1]
+  int64_t rows_alloc;      // rows of the grouped buffers
+  int n_tiles;             // N / BN
+  int m_tiles;             // kWG: M / BM
+  int num_kb;              // kDH: d / BK;  kDX: 2 f / BK
+  int half_kb;             // kDX: f / BK (first half dG x W_gate, second dU x W_up)
+  int m_outer;             // kWG: tiles of one expert ordered M-block major
+  const int32_t* perm;     // kDX: token of each row
+  int64_t n_tok;
+  const float* row_scale;  // kDH
+  const __nv_bfloat16* G;  // kDH inputs [rows, f]
+  const __nv_bfloat16* U;
+  const __nv_bfloat16* H;
+  __nv_bfloat16* dG;       // kDH outputs [rows, f]
+  __nv_bfloat16* dU;
+  float* dw_part;          // kDH: [rows, n_tiles]
+  float* out;              // kDX: dx32 [T, d];  kWG: dW [E, M, N]
+  int64_t ld;              // kDH: f;  kDX: d;  kWG: N
+  int64_t M;               // kWG
+  int* err;
+};
+
+struct Sched {
+  int offs[kE + 1];
+  int mt[kE];              // row blocks (kDH, kDX) of each expert
+  int prefix[kE + 1];
+};
+
+struct Tile {
+  int e, m0, rows, n0, nb;
+  int row0, nrows, nkb;    // kWG: the expert's grouped rows and K blocks
+};
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(const Sched& s, const BwdArgs& a, int L) {
+  Tile t;
+  int e = 0;
+#pragma unroll
+  for (int k = 1; k < kE; ++k)
+    if (L >= s.prefix[k]) e = k;
+  const int local = L - s.prefix[e];
+  t.e = e;
+  t.row0 = s.offs[e];
+  t.nrows = s.offs[e + 1] - s.offs[e];
+  if (MODE == kWG) {
+    int mb, nb;
+    if (a.m_outer) {
+      mb = local / a.n_tiles;
+      nb = local - mb * a.n_tiles;
+    } else {
+      nb = local / a.m_tiles;
+      mb = local - nb * a.m_tiles;
+    }
+    t.m0 = mb * BM;
+    t.rows = BM;
+    t.n0 = nb * BN;
+    t.nb = nb;
+    t.nkb = (t.nrows + BK - 1) / BK;
+  } else {
+    const int nb = local / s.mt[e];
+    const int mi = local - nb * s.mt[e];
+    t.m0 = s.offs[e] + mi * BM;
+    const int left = s.offs[e + 1] - t.m0;
+    t.rows = left < BM ? left : BM;
+    t.n0 = nb * BN;
+    t.nb = nb;
+    t.nkb = MODE == kDH ? a.num_kb : 2 * a.half_kb;
+  }
+  return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ void build_schedule(Sched& sched, const BwdArgs& args) {
+  bool ok = true;
+  int prev = 0;
+  for (int k = 0; k <= kE; ++k) {
+    const int v = args.offsets[k];
+    sched.offs[k] = v;
+    if (v < prev || (int64_t)v > args.rows_alloc) ok = false;
+    prev = v;
+  }
+  if (sched.offs[0] < 0) ok = false;
+  if (!ok)
+    for (int k = 0; k <= kE; ++k) sched.offs[k] = 0;
+  int acc = 0;
+  for (int k = 0; k < kE; ++k) {
+    const int n = sched.offs[k + 1] - sched.offs[k];
+    sched.mt[k] = (n + BM - 1) / BM;
+    sched.prefix[k] = acc;
+    // weight gradients: every expert owns its M x N tiles (zero when it has no rows)
+    acc += MODE == kWG ? (ok ? args.m_tiles * args.n_tiles : 0) : sched.mt[k] * args.n_tiles;
+  }
+  sched.prefix[kE] = acc;
+  if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
+}
+
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                    const BwdArgs args) {
+  constexpr int S = kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * STAGE);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ Sched sched;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 1) {
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmB0);
+    if (MODE == kDX) {
+      prefetch_tmap(&tmA1);
+      prefetch_tmap(&tmB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 2 && lane == 0) build_schedule<MODE>(sched, args);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = sched.prefix[kE];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t it = 0;
+      bool ok = true;
+      const uint64_t keep = policy_evict_last();
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        const Tile t = decode_tile<MODE>(sched, args, L);
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], STAGE);
+          uint8_t* a = sA + s * A_BYTES;
+          uint8_t* b = sB + s * B_BYTES;
+          if (MODE == kDH) {
+            tma_load_2d_hint(a, &tmA0, &full[s], kb * BK, t.m0, keep);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tma_load_3d_hint(b + c * CHUNK, &tmB0, &full[s], kb * BK, t.n0 + 64 * c, t.e, keep);
+          } else if (MODE == kDX) {
+            const bool first = kb < args.half_kb;
+            const int k0 = (first ? kb : kb - args.half_kb) * BK;
+            tma_load_2d_hint(a, first ? &tmA0 : &tmA1, &full[s], k0, t.m0, keep);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_3d_hint(b + c * CHUNK, first ? &tmB0 : &tmB1, &full[s], k0, t.n0 + 64 * c, t.e, keep);
+          } else {
+            const int r0 = t.row0 + kb * BK;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) tma_load_2d_hint(a + c * CHUNK, &tmA0, &full[s], t.m0 + 64 * c, r0, keep);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tma_load_2d_hint(b + c * CHUNK, &tmB0, &full[s], t.n0 + 64 * c, r0, keep);
+          }
+        }
+      }
+      if (!ok) {
+        flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      const uint32_t first = it > (uint32_t)S ? it - S : 0u;
+      for (uint32_t j = first; j < it; ++j) mbar_wait(&full[j % S], (j / S) & 1u, nullptr, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    // Lane 0 waits and issues; for the weight gradients all 32 lanes zero the
+    // rows past the expert's end in its last K block first.
+    constexpr bool kMN = MODE == kWG;
+    constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kMN, kMN);
+    uint32_t it = 0, tc = 0;
+    bool ok = true, issued = false;
+    for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+      const Tile t = decode_tile<MODE>(sched, args, L);
+      const uint32_t buf = tc & 1u;
+      const uint32_t tph = (tc >> 1) & 1u;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&tempty[buf], tph ^ 1u, abort_flag) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + buf * kAccStride;
+      for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        // weight gradients: every lane observes the landed stage itself, since
+        // lanes may overwrite part of it below
+        if (lane == 0 || MODE == kWG) got = mbar_wait(&full[s], ph, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        if (MODE == kWG) {
+          const int valid = t.nrows - kb * BK;
+          if (valid < BK) {
+            // rows [valid, 64) of the 6 chunks (2 of A, 4 of B) belong to the next
+            // expert or lie past the kept rows: zero them (each row is 128 bytes)
+            uint8_t* base = sA + s * A_BYTES;
+            const int per_chunk = (BK - valid) * 8;  // 16-byte pieces
+            for (int i = lane; i < 6 * per_chunk; i += 32) {
+              const int c = i / per_chunk;
+              const int j = i - c * per_chunk;
+              uint8_t* chunk = c < 2 ? base + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
+              *reinterpret_cast<uint4*>(chunk + valid * 128 + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            uint64_t ad, bd;
+            if (kMN) {
+              ad = sw128_desc(a_addr + kk * 2048, CHUNK, 1024);
+              bd = sw128_desc(b_addr + kk * 2048, CHUNK, 1024);
+            } else {
+              ad = sw128_desc(a_addr + kk * 32, 16, 1024);
+              bd = sw128_desc(b_addr + kk * 32, 16, 1024);
+            }
+            umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(&empty[s]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&tfull[buf]);
+    }
+    if (lane == 0) {
+      if (!ok) {
+        flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (issued) {
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, 100000000ull);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    uint32_t tc = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
+      const Tile t = decode_tile<MODE>(sched, args, L);
+      const uint32_t buf = tc & 1u;
+      const uint32_t tph = (tc >> 1) & 1u;
+      if (!mbar_wait(&tfull[buf], tph, abort_flag)) {
+        if (lane == 0) flag_error(args.err, MOE_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + buf * kAccStride + ((uint32_t)(q * 32) << 16);
+      if (MODE == kDH) {
+        const bool valid = r < t.rows;
+        const int64_t row = t.m0 + r;
+        const float w = valid ? __ldg(args.row_scale + row) : 0.f;
+        const int64_t base = row * args.ld + t.n0;
+        float dot = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int64_t o = base + c * 32 + p * 8;
+              float g[8], u[8], h[8];
+              load8_bf16(args.G + o, g);
+              load8_bf16(args.U + o, u);
+              load8_bf16(args.H + o, h);
+              uint32_t og[4], ou[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                float dg2[2], du2[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                  const int j = 2 * i + k;
+                  const float dhu = __uint_as_float(v[p * 8 + j]);
+                  dot = fmaf(dhu, h[j], dot);
+                  const float dh = w * dhu;
+                  const float sg = 1.0f / (1.0f + __expf(-g[j]));
+                  const float sl = g[j] * sg;
+                  dg2[k] = dh * u[j] * (sg * (1.0f + g[j] * (1.0f - sg)));
+                  du2[k] = dh * sl;
+                }
+                og[i] = pack_bf16x2(dg2[0], dg2[1]);
+                ou[i] = pack_bf16x2(du2[0], du2[1]);
+              }
+              *reinterpret_cast<uint4*>(args.dG + o) = make_uint4(og[0], og[1], og[2], og[3]);
+              *reinterpret_cast<uint4*>(args.dU + o) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+            }
+          }
+        }
+        if (valid) args.dw_part[row * args.n_tiles + t.nb] = dot;
+      } else if (MODE == kDX) {
+        int tok = -1;
+        if (r < t.rows) {
+          tok = __ldg(args.perm + t.m0 + r);
+          if (tok < 0 || (int64_t)tok >= args.n_tok) {
+            flag_error(args.err, MOE_DEVERR_SLOT_INDEX);
+            tok = -1;
+          }
+        }
+        float* dst = args.out + (int64_t)(tok < 0 ? 0 : tok) * args.ld + t.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          if (tok >= 0) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              atomicAdd(d4 + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
+          }
+        }
+      } else {
+        float* dst = args.out + ((int64_t)t.e * args.M + t.m0 + r) * args.ld + t.n0;
+        const bool zero = t.nkb == 0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                         : make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int MODE>
+cudaError_t launch_bwd(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const BwdArgs& args, cudaStream_t s, const Ctx& ctx) {
+  auto kern = bwd_gemm_kernel<MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<ctx.num_sms, kThreads, SMEM_BYTES, s>>>(a0, a1, b0, b1, args);
+  return cudaGetLastError();
+}
+
+BwdArgs base_args(const moe_config_t& c, const int32_t* offsets, const Ctx& ctx) {
+  BwdArgs a = {};
+  a.offsets = offsets;
+  a.rows_alloc = slot_rows(c);
+  a.n_tok = c.T;
+  a.err = ctx.err;
+  return a;
+}
+
+bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t str[1] = {(uint64_t)cols * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return encode_tmap(m, base, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// [E, R, C] weights, box of 64 columns x 64 rows of one expert
+bool map_weights(CUtensorMap* m, const void* base, int E, int64_t R, int64_t C) {
+  const uint64_t dims[3] = {(uint64_t)C, (uint64_t)R, (uint64_t)E};
+  const uint64_t str[2] = {(uint64_t)C * 2, (uint64_t)R * C * 2};
+  const uint32_t box[3] = {64, 64, 1};
+  return encode_tmap(m, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dh(const moe_config_t& c, const void* dout_perm, const int32_t* offsets, const void* wd,
+                          const void* G, const void* U, const void* H, const float* row_scale, void* dG, void* dU,
+                          float* dw_part, cudaStream_t s, const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap ta, tb;
+  // W_down [E, f, d] read K-major: rows = f (N), columns = d (K)
+  if (!map_rows(&ta, dout_perm, rows, c.d, 128) || !map_weights(&tb, wd, c.E, c.f, c.d))
+    return cudaErrorInvalidValue;
+  BwdArgs a = base_args(c, offsets, ctx);
+  a.n_tiles = (int)(c.f / BN);
+  a.num_kb = (int)(c.d / BK);
+  a.row_scale = row_scale;
+  a.G = static_cast<const __nv_bfloat16*>(G);
+  a.U = static_cast<const __nv_bfloat16*>(U);
+  a.H = static_cast<const __nv_bfloat16*>(H);
+  a.dG = static_cast<__nv_bfloat16*>(dG);
+  a.dU = static_cast<__nv_bfloat16*>(dU);
+  a.dw_part = dw_part;
+  a.ld = c.f;
+  return launch_bwd<kDH>(ta, ta, tb, tb, a, s, ctx);
+}
+
+cudaError_t launch_bwd_dx(const moe_config_t& c, const void* dG, const void* dU, const int32_t* offsets,
+                          const void* wg, const void* wu, const int32_t* perm, float* dx32, cudaStream_t s,
+                          const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap ta0, ta1, tb0, tb1;
+  // W_gate / W_up [E, d, f] read K-major: rows = d (N), columns = f (K)
+  if (!map_rows(&ta0, dG, rows, c.f, 128) || !map_rows(&ta1, dU, rows, c.f, 128) ||
+      !map_weights(&tb0, wg, c.E, c.d, c.f) || !map_weights(&tb1, wu, c.E, c.d, c.f))
+    return cudaErrorInvalidValue;
+  BwdArgs a = base_args(c, offsets, ctx);
+  a.n_tiles = (int)(c.d / BN);
+  a.half_kb = (int)(c.f / BK);
+  a.num_kb = 2 * a.half_kb;
+  a.perm = perm;
+  a.out = dx32;
+  a.ld = c.d;
+  return launch_bwd<kDX>(ta0, ta1, tb0, tb1, a, s, ctx);
+}
+
+cudaError_t launch_bwd_wgrad(const moe_config_t& c, const void* a_rows, int64_t M, const void* b_rows, int64_t N,
+                             const int32_t* offsets, float* dW, bool m_outer, cudaStream_t s, const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0 || M % BM != 0 || N % BN != 0) return rows == 0 ? cudaSuccess : cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!map_rows(&ta, a_rows, rows, M, 64) || !map_rows(&tb, b_rows, rows, N, 64)) return cudaErrorInvalidValue;
+  BwdArgs a = base_args(c, offsets, ctx);
+  a.m_tiles = (int)(M / BM);
+  a.n_tiles = (int)(N / BN);
+  a.m_outer = m_outer ? 1 : 0;
+  a.out = dW;
+  a.ld = N;
+  a.M = M;
+  return launch_bwd<kWG>(ta, ta, tb, tb, a, s, ctx);
+}
+
+}  // namespace moe

@@ -72,6 +72,10 @@ struct TcArgs {
   void* out;
   int64_t ld_out;          // elements per output row
   const float* row_scale;  // down only; NULL means 1
+  const int32_t* perm;     // fused variants: source token of each row
+  int64_t n_tok;           // fused variants: rows of x / out (tokens)
+  void* save_g;            // gate/up for training: also write G and U (bf16) or NULL
+  void* save_u;
   int* err;
 };
 
@@ -127,11 +131,29 @@ __device__ __forceinline__ void build_schedule(Sched& sched, const TcArgs& args,
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <int MODE, int MMA_N>
+// Source token of grouped row `row` for the fused variants (0 for rows past the
+// kept ones, which are computed and never stored; a bad index is flagged).
+__device__ __forceinline__ int source_token(const TcArgs& args, int row, int n_rows) {
+  if (row >= n_rows) return 0;
+  const int t = __ldg(args.perm + row);
+  if (t < 0 || (int64_t)t >= args.n_tok) {
+    flag_error(args.err, MOE_DEVERR_SLOT_INDEX);
+    return -1;
+  }
+  return t;
+}
+
+// FUSED = true (down only): instead of writing Y by grouped row, the epilogue
+// adds row_scale * (H W_down) into a zeroed fp32 out[token] with vector
+// atomics.  With top-2 a token receives at most two terms and 0 + a + b rounds
+// the same in either order, so the result is the combine's fp32 sum bit for
+// bit, without the Y buffer.
+template <int MODE, int MMA_N, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                            const __grid_constant__ CUtensorMap tmB1, const TcArgs args) {
   using C = Cfg<MODE, MMA_N>;
+  constexpr bool kScatter = FUSED && MODE == kDown;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -299,6 +321,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            if (args.save_g) {
+              // training: keep the pre-activations for the backward pass
+              const int64_t o = (int64_t)(t.m0 + r) * args.ld_out + t.n0 + c * 32;
+              uint4* g4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.save_g) + o);
+              uint4* u4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.save_u) + o);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                g4[i] = make_uint4(pack_bf16x2(__uint_as_float(g[8 * i]), __uint_as_float(g[8 * i + 1])),
+                                   pack_bf16x2(__uint_as_float(g[8 * i + 2]), __uint_as_float(g[8 * i + 3])),
+                                   pack_bf16x2(__uint_as_float(g[8 * i + 4]), __uint_as_float(g[8 * i + 5])),
+                                   pack_bf16x2(__uint_as_float(g[8 * i + 6]), __uint_as_float(g[8 * i + 7])));
+                u4[i] = make_uint4(pack_bf16x2(__uint_as_float(u[8 * i]), __uint_as_float(u[8 * i + 1])),
+                                   pack_bf16x2(__uint_as_float(u[8 * i + 2]), __uint_as_float(u[8 * i + 3])),
+                                   pack_bf16x2(__uint_as_float(u[8 * i + 4]), __uint_as_float(u[8 * i + 5])),
+                                   pack_bf16x2(__uint_as_float(u[8 * i + 6]), __uint_as_float(u[8 * i + 7])));
+              }
+            }
+          }
+        }
+      } else if (kScatter) {
+        float* O = static_cast<float*>(args.out);
+        const int tok = valid ? source_token(args, t.m0 + r, sched.offs[kE]) : -1;
+        const bool store = tok >= 0;
+        float* dst_row = O + (int64_t)(store ? tok : 0) * args.ld_out + t.n0;
+        const float sc = (store && args.row_scale) ? __ldg(args.row_scale + t.m0 + r) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < C::BN_OUT / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + c * 32, v);
+          tmem_wait_ld();
+          if (store) {
+            float4* d4 = reinterpret_cast<float4*>(dst_row + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              atomicAdd(d4 + i, make_float4(sc * __uint_as_float(v[4 * i]), sc * __uint_as_float(v[4 * i + 1]),
+                                            sc * __uint_as_float(v[4 * i + 2]), sc * __uint_as_float(v[4 * i + 3])));
           }
         }
       } else {
@@ -331,11 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int MODE, int MMA_N>
+template <int MODE, int MMA_N, bool FUSED = false>
 cudaError_t launch_grouped(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const TcArgs& args,
                            cudaStream_t s, const Ctx& ctx) {
   using C = Cfg<MODE, MMA_N>;
-  auto kern = grouped_gemm_tc_kernel<MODE, MMA_N>;
+  auto kern = grouped_gemm_tc_kernel<MODE, MMA_N, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<ctx.num_sms, kThreads, C::SMEM_BYTES, s>>>(a, b0, b1, args);
@@ -345,7 +403,8 @@ cudaError_t launch_grouped(const CUtensorMap& a, const CUtensorMap& b0, const CU
 }  // namespace
 
 cudaError_t launch_tc_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
-                              const void* wg, const void* wu, void* h, cudaStream_t s, const Ctx& ctx) {
+                              const void* wg, const void* wu, void* h, cudaStream_t s, const Ctx& ctx, void* g_save,
+                              void* u_save) {
   const int64_t rows = slot_rows(c);
   if (rows == 0) return cudaSuccess;
   CUtensorMap ta, tg, tu;
@@ -367,6 +426,10 @@ cudaError_t launch_tc_gate_up(const moe_config_t& c, const void* x_perm, const i
   args.out = h;
   args.ld_out = c.f;
   args.row_scale = nullptr;
+  args.perm = nullptr;
+  args.n_tok = c.T;
+  args.save_g = g_save;
+  args.save_u = u_save;
   args.err = ctx.err;
   return launch_grouped<kGateUp, 256>(ta, tg, tu, args, s, ctx);
 }
@@ -392,6 +455,10 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
   args.out = y;
   args.ld_out = c.d;
   args.row_scale = row_scale;
+  args.perm = nullptr;
+  args.n_tok = c.T;
+  args.save_g = nullptr;
+  args.save_u = nullptr;
   args.err = ctx.err;
   if (c.d % 256 == 0) {
     args.n_tiles = (int)(c.d / 256);
@@ -399,6 +466,38 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
   }
   args.n_tiles = (int)(c.d / 128);
   return launch_grouped<kDown, 128>(ta, tw, tw, args, s, ctx);
+}
+
+cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
+                                   const float* row_scale, const int32_t* perm, float* out32, cudaStream_t s,
+                                   const Ctx& ctx) {
+  const int64_t rows = slot_rows(c);
+  if (rows == 0) return cudaSuccess;
+  if (c.d % 256 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tw;
+  const uint64_t a_dims[2] = {(uint64_t)c.f, (uint64_t)rows};
+  const uint64_t a_str[1] = {(uint64_t)c.f * 2};
+  const uint32_t a_box[2] = {64, 128};
+  const uint64_t w_dims[3] = {(uint64_t)c.d, (uint64_t)c.f, (uint64_t)c.E};
+  const uint64_t w_str[2] = {(uint64_t)c.d * 2, (uint64_t)c.f * c.d * 2};
+  const uint32_t w_box[3] = {64, 64, 1};
+  if (!encode_tmap(&ta, h, 2, a_dims, a_str, a_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tw, wd, 3, w_dims, w_str, w_box, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  TcArgs args;
+  args.offsets = offsets;
+  args.rows_alloc = rows;
+  args.num_kb = (int)(c.f / BK);
+  args.out = out32;
+  args.ld_out = c.d;
+  args.row_scale = row_scale;
+  args.perm = perm;
+  args.n_tok = c.T;
+  args.save_g = nullptr;
+  args.save_u = nullptr;
+  args.err = ctx.err;
+  args.n_tiles = (int)(c.d / 256);
+  return launch_grouped<kDown, 256, true>(ta, tw, tw, args, s, ctx);
 }
 
 }  // namespace moe

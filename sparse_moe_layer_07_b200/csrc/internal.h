@@ -49,12 +49,45 @@ cudaError_t launch_ffn_simt_down(const moe_config_t& c, const float* h, const in
                                  cudaStream_t s, const Ctx& ctx);
 
 // bf16 expert FFN on the tcgen05 tensor cores.
+// g_save / u_save (training): also write the pre-activations G, U [T*k, f] (bf16).
 cudaError_t launch_tc_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
                               const void* wg, const void* wu, void* h, cudaStream_t s,
-                              const Ctx& ctx);
+                              const Ctx& ctx, void* g_save = nullptr, void* u_save = nullptr);
 cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* offsets,
                            const void* wd, const float* row_scale, float* y, cudaStream_t s,
                            const Ctx& ctx);
+
+// Down with the combine fused: adds row_scale * (H W_down) into a zeroed fp32
+// out32 [T, d] by token (perm) instead of writing Y.
+cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
+                                   const float* row_scale, const int32_t* perm, float* out32, cudaStream_t s,
+                                   const Ctx& ctx);
+// Backward of the expert FFNs (bf16, d and f multiples of 256): dG / dU and the
+// routing-weight partials, dx (added into a zeroed fp32 dx32 by token), and
+// the weight gradients dW[e] = A_e^T B_e over each expert's rows ([E, M, N] fp32).
+cudaError_t launch_bwd_dh(const moe_config_t& c, const void* dout_perm, const int32_t* offsets, const void* wd,
+                          const void* G, const void* U, const void* H, const float* row_scale, void* dG, void* dU,
+                          float* dw_part, cudaStream_t s, const Ctx& ctx);
+cudaError_t launch_bwd_dx(const moe_config_t& c, const void* dG, const void* dU, const int32_t* offsets,
+                          const void* wg, const void* wu, const int32_t* perm, float* dx32, cudaStream_t s,
+                          const Ctx& ctx);
+cudaError_t launch_bwd_wgrad(const moe_config_t& c, const void* a_rows, int64_t M, const void* b_rows, int64_t N,
+                             const int32_t* offsets, float* dW, bool m_outer, cudaStream_t s, const Ctx& ctx);
+// dout_perm[r] = dout[perm[r]],  dy_perm[r] = bf16(row_scale[r] * dout[perm[r]])  (r < offsets[E])
+cudaError_t launch_bwd_gather(const moe_config_t& c, const void* dout, const int32_t* perm, const int32_t* offsets,
+                              const float* row_scale, void* dout_perm, void* dy_perm, cudaStream_t s, const Ctx& ctx);
+// Router backward: routing-weight gradients from the partials, logit gradients
+// through the softmax over the two selected logits, dx = round(dx32 + dlogits W_r),
+// dW_r = dlogits^T x and dbias = column sums of dlogits (fixed summation orders).
+cudaError_t launch_router_bwd(const moe_config_t& c, const float* dw_part, int n_parts, const int32_t* slot_of,
+                              const int32_t* topk_idx, const float* topk_w, const void* w_router, const float* dx32,
+                              const void* x, float* dlogits, float* dweight, void* dx, float* dw_router,
+                              float* dbias, float* wr_part, cudaStream_t s, const Ctx& ctx);
+constexpr int kRouterBwdChunks = 32;  // token chunks of the dW_r partial sums
+
+// out32 <- 0 ([T, d] fp32), and out <- out32 rounded to cfg's dtype.
+cudaError_t launch_zero_rows(const moe_config_t& c, float* out32, cudaStream_t s, const Ctx& ctx);
+cudaError_t launch_round_out(const moe_config_t& c, const float* out32, void* out, cudaStream_t s, const Ctx& ctx);
 
 // Argument check shared by the entry points (MOE_OK when the config is usable).
 moe_status_t validate_config(const moe_config_t* cfg);

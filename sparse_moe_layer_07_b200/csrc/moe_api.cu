@@ -127,6 +127,12 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 // the MMA's M side and spends no tensor time on padded token rows.
 bool weight_streaming(const moe_config_t& c) { return c.T * (int64_t)c.top_k <= 64 * (int64_t)c.E; }
 
+// The one-call bf16 layer with row-major tensor-core tiles runs the down pass
+// with the combine fused (the Y region holds the fp32 sums: T*d <= T*k*d).
+bool fused_layer(const moe_config_t& c) {
+  return c.dtype == MOE_BF16 && !weight_streaming(c) && c.d % 256 == 0 && c.top_k == 2;
+}
+
 moe_status_t run_gate_up(const moe_config_t& c, const void* x_perm, const int32_t* offsets, const void* wg,
                          const void* wu, void* h, cudaStream_t s, const Ctx& ctx) {
   if (c.dtype == MOE_BF16 && weight_streaming(c))
@@ -278,6 +284,32 @@ moe_status_t moe_expert_down(const moe_config_t* cfg, const void* h, const int32
   return run_down(*cfg, h, offsets, w_down, row_scale, y, stream, ctx);
 }
 
+size_t moe_expert_down_combine_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return round_up((size_t)cfg->T * cfg->d * 4);
+}
+
+moe_status_t moe_expert_down_combine(const moe_config_t* cfg, const void* h, const int32_t* offsets,
+                                     const void* w_down, const float* row_scale, const int32_t* perm, void* out,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!fused_layer(*cfg)) return MOE_ERR_UNSUPPORTED;
+  if (!h || !offsets || !w_down || !perm || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down) || !aligned16(out) || (row_scale && !aligned16(row_scale)))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_expert_down_combine_workspace_size(cfg)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  float* out32 = static_cast<float*>(ws);
+  cudaError_t e = launch_zero_rows(*cfg, out32, stream, ctx);
+  if (e == cudaSuccess) e = launch_tc_down_scatter(*cfg, h, offsets, w_down, row_scale, perm, out32, stream, ctx);
+  if (e == cudaSuccess) e = launch_round_out(*cfg, out32, out, stream, ctx);
+  return cuda_status(e);
+}
+
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate,
                             const void* w_up, const void* w_down, const float* row_scale, void* h, float* y, void* ws,
                             size_t ws_bytes, moe_stream_t stream) {
@@ -324,6 +356,16 @@ static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, con
                         row_scale, disp, stats, s, ctx);
   if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, x_perm, s, ctx);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (fused_layer(c)) {
+    // down accumulates straight into out32 by token (in the Y region, which this
+    // path does not use); one rounding pass writes out
+    float* out32 = y;
+    e = launch_zero_rows(c, out32, s, ctx);
+    if (e == cudaSuccess) e = launch_tc_gate_up(c, x_perm, offsets, w_gate, w_up, h, s, ctx);
+    if (e == cudaSuccess) e = launch_tc_down_scatter(c, h, offsets, w_down, row_scale, perm, out32, s, ctx);
+    if (e == cudaSuccess) e = launch_round_out(c, out32, out, s, ctx);
+    return cuda_status(e);
+  }
   moe_status_t st = run_gate_up(c, x_perm, offsets, w_gate, w_up, h, s, ctx);
   if (st == MOE_OK) st = run_down(c, h, offsets, w_down, row_scale, y, s, ctx);
   if (st == MOE_OK) st = cuda_status(launch_combine(c, y, slot_of, topk_w, 1, out, s, ctx));
@@ -378,6 +420,77 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
   if (cudaMemcpyAsync(out_host, w8 + L.out, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(cudaStreamSynchronize(stream));
+}
+
+size_t moe_workspace_size_host_batches(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg).total + 2 * round_up((size_t)cfg->T * cfg->d * esize(*cfg));
+}
+
+// Two-slot copy/compute pipeline: batch i uses staging slot i % 2 (x and out).
+//   h2d stream : wait comp[s] (batch i-2 done with slot s), copy x_host[i] -> x slot, record xin[s]
+//   stream     : wait xin[s] and outfree[s] (batch i-2's result copied out), layer, record comp[s]
+//   d2h stream : wait comp[s], copy out slot -> out_host[i], record outfree[s]
+// Enqueued in that order for each i, so batch i+1's copy-in and batch i-1's
+// copy-out run while batch i computes.  cudaStreamWaitEvent binds the event's
+// latest record at enqueue time, which is always the batch two steps back.
+moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_batches, const void* const* x_host,
+                                            const void* w_router, const float* logit_bias, const void* w_gate,
+                                            const void* w_up, const void* w_down, void* const* out_host, void* ws,
+                                            size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (n_batches < 0) return MOE_ERR_INVALID_ARG;
+  if (n_batches == 0 || cfg->T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < n_batches; ++i)
+    if (!x_host[i] || !out_host[i]) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size_host_batches(cfg)) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  const Layout L = layout_of(c);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const size_t bytes = (size_t)c.T * c.d * esize(c);
+  uint8_t* x_slot[2] = {w8 + L.x_in, w8 + L.total};
+  uint8_t* out_slot[2] = {w8 + L.out, w8 + L.total + round_up(bytes)};
+
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev[7] = {};  // start, xin[2], comp[2], outfree[2]
+  cudaEvent_t &start = ev[0], *xin = ev + 1, *comp = ev + 3, *outfree = ev + 5;
+  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; ok && i < 7; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  // the whole pipeline starts after the work already in `stream`
+  ok = ok && cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(h2d, start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(d2h, start, 0) == cudaSuccess;
+  for (int64_t i = 0; ok && i < n_batches; ++i) {
+    const int sl = (int)(i & 1);
+    if (i >= 2) ok = cudaStreamWaitEvent(h2d, comp[sl], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(x_slot[sl], x_host[i], bytes, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaEventRecord(xin[sl], h2d) == cudaSuccess && cudaStreamWaitEvent(stream, xin[sl], 0) == cudaSuccess;
+    if (ok && i >= 2) ok = cudaStreamWaitEvent(stream, outfree[sl], 0) == cudaSuccess;
+    if (!ok) break;
+    st = layer_forward_impl(c, x_slot[sl], w_router, logit_bias, w_gate, w_up, w_down, out_slot[sl], nullptr, w8,
+                            stream, ctx);
+    if (st != MOE_OK) break;
+    ok = cudaEventRecord(comp[sl], stream) == cudaSuccess && cudaStreamWaitEvent(d2h, comp[sl], 0) == cudaSuccess &&
+         cudaMemcpyAsync(out_host[i], out_slot[sl], bytes, cudaMemcpyDeviceToHost, d2h) == cudaSuccess &&
+         cudaEventRecord(outfree[sl], d2h) == cudaSuccess;
+  }
+  // later work in `stream` is ordered after the last copy-out; then wait for all of it
+  if (ok && st == MOE_OK) ok = cudaEventRecord(start, d2h) == cudaSuccess && cudaStreamWaitEvent(stream, start, 0) == cudaSuccess;
+  cudaError_t sync = cudaSuccess;
+  if (d2h) sync = cudaStreamSynchronize(d2h);
+  if (h2d && sync == cudaSuccess) sync = cudaStreamSynchronize(h2d);
+  if (sync == cudaSuccess) sync = cudaStreamSynchronize(stream);
+  for (int i = 0; i < 7; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);
+  if (h2d) cudaStreamDestroy(h2d);
+  if (d2h) cudaStreamDestroy(d2h);
+  if (st != MOE_OK) return st;
+  if (!ok) return MOE_ERR_CUDA;
+  return cuda_status(sync);
 }
 
 moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
@@ -535,6 +648,152 @@ moe_status_t moe_get_device_error(int32_t* code, int32_t clear) {
   }
   *code = v;
   return v ? MOE_ERR_DEVICE_CHECK : MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------- training
+namespace moe {
+namespace {
+
+// Workspace of the training pair: the forward's layout, then what the backward
+// reads (G, U) and its own scratch.
+struct TrainLayout {
+  Layout base;
+  size_t g, u, dout_perm, dy_perm, dg, du, dw_part, dlogits, dweight, dx32, wr_part, total;
+};
+
+TrainLayout train_layout_of(const moe_config_t& c) {
+  TrainLayout L;
+  L.base = layout_of(c);
+  const size_t rows = (size_t)slot_rows(c);
+  size_t o = L.base.total;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += round_up(bytes);
+    return at;
+  };
+  L.g = take(rows * c.f * 2);
+  L.u = take(rows * c.f * 2);
+  L.dout_perm = take(rows * c.d * 2);
+  L.dy_perm = take(rows * c.d * 2);
+  L.dg = take(rows * c.f * 2);
+  L.du = take(rows * c.f * 2);
+  L.dw_part = take(rows * (size_t)(c.f / 256) * 4);
+  L.dlogits = take((size_t)c.T * c.E * 4);
+  L.dweight = take((size_t)c.T * c.top_k * 4);
+  L.dx32 = take((size_t)c.T * c.d * 4);
+  L.wr_part = take((size_t)kRouterBwdChunks * c.E * c.d * 4);
+  L.total = o;
+  return L;
+}
+
+bool train_supported(const moe_config_t& c) {
+  return c.dtype == MOE_BF16 && c.d % 256 == 0 && c.f % 256 == 0 && c.top_k == 2;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_workspace_size_train(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK || !train_supported(*cfg)) return 0;
+  return train_layout_of(*cfg).total;
+}
+
+moe_status_t moe_layer_forward_train(const moe_config_t* cfg, const void* x, const void* w_router,
+                                     const float* logit_bias, const void* w_gate, const void* w_up,
+                                     const void* w_down, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (!train_supported(*cfg)) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size_train(cfg)) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  const TrainLayout TL = train_layout_of(c);
+  const Layout& L = TL.base;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(w8 + L.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(w8 + L.topk_w);
+  int32_t* route = reinterpret_cast<int32_t*>(w8 + L.route);
+  int32_t* offsets = route + 2 * c.E;
+  int32_t* perm = reinterpret_cast<int32_t*>(w8 + L.perm);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(w8 + L.slot_of);
+  float* row_scale = reinterpret_cast<float*>(w8 + L.row_scale);
+  float* y = reinterpret_cast<float*>(w8 + L.y);
+  cudaError_t e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, route, route + c.E, offsets, perm, slot_of, row_scale,
+                        reinterpret_cast<int32_t*>(w8 + L.disp), nullptr, stream, ctx);
+  if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, w8 + L.x_perm, stream, ctx);
+  // the row-major tensor-core kernels at every batch size: gate/up keeps G and U
+  if (e == cudaSuccess)
+    e = launch_tc_gate_up(c, w8 + L.x_perm, offsets, w_gate, w_up, w8 + L.h, stream, ctx, w8 + TL.g, w8 + TL.u);
+  if (e == cudaSuccess) e = launch_tc_down(c, w8 + L.h, offsets, w_down, row_scale, y, stream, ctx);
+  if (e == cudaSuccess) e = launch_combine(c, y, slot_of, topk_w, 1, out, stream, ctx);
+  return cuda_status(e);
+}
+
+moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const void* w_router, const void* w_gate,
+                                const void* w_up, const void* w_down, const void* dout, void* dx, float* dw_router,
+                                float* dbias, float* dw_gate, float* dw_up, float* dw_down, void* ws,
+                                size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(cfg, w_router, nullptr, w_gate, w_up, w_down, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (!train_supported(*cfg)) return MOE_ERR_UNSUPPORTED;
+  if (!dw_router || !dw_gate || !dw_up || !dw_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dw_router) || !aligned16(dw_gate) || !aligned16(dw_up) || !aligned16(dw_down) ||
+      (dbias && !aligned16(dbias)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!x || !dout || !dx || !aligned16(x) || !aligned16(dout) || !aligned16(dx)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && ws_bytes < moe_workspace_size_train(cfg)) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T == 0) {
+    // no tokens: every gradient is zero
+    cudaError_t e = cudaMemsetAsync(dw_router, 0, (size_t)c.E * c.d * 4, stream);
+    if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, (size_t)c.E * 4, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_gate, 0, (size_t)c.E * c.d * c.f * 4, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_up, 0, (size_t)c.E * c.d * c.f * 4, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_down, 0, (size_t)c.E * c.d * c.f * 4, stream);
+    return cuda_status(e);
+  }
+  const TrainLayout TL = train_layout_of(c);
+  const Layout& L = TL.base;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int32_t* topk_idx = reinterpret_cast<const int32_t*>(w8 + L.topk_idx);
+  const float* topk_w = reinterpret_cast<const float*>(w8 + L.topk_w);
+  const int32_t* offsets = reinterpret_cast<const int32_t*>(w8 + L.route) + 2 * c.E;
+  const int32_t* perm = reinterpret_cast<const int32_t*>(w8 + L.perm);
+  const int32_t* slot_of = reinterpret_cast<const int32_t*>(w8 + L.slot_of);
+  const float* row_scale = reinterpret_cast<const float*>(w8 + L.row_scale);
+  float* dw_part = reinterpret_cast<float*>(w8 + TL.dw_part);
+  float* dx32 = reinterpret_cast<float*>(w8 + TL.dx32);
+  const int n_parts = (int)(c.f / 256);
+  cudaError_t e = launch_bwd_gather(c, dout, perm, offsets, row_scale, w8 + TL.dout_perm, w8 + TL.dy_perm, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_bwd_dh(c, w8 + TL.dout_perm, offsets, w_down, w8 + TL.g, w8 + TL.u, w8 + L.h, row_scale, w8 + TL.dg,
+                      w8 + TL.du, dw_part, stream, ctx);
+  if (e == cudaSuccess) e = launch_zero_rows(c, dx32, stream, ctx);
+  if (e == cudaSuccess) e = launch_bwd_dx(c, w8 + TL.dg, w8 + TL.du, offsets, w_gate, w_up, perm, dx32, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_router_bwd(c, dw_part, n_parts, slot_of, topk_idx, topk_w, w_router, dx32, x,
+                          reinterpret_cast<float*>(w8 + TL.dlogits), reinterpret_cast<float*>(w8 + TL.dweight), dx,
+                          dw_router, dbias, reinterpret_cast<float*>(w8 + TL.wr_part), stream, ctx);
+  // weight gradients: the larger operand's blocks outermost, so the smaller one stays in L2
+  if (e == cudaSuccess)
+    e = launch_bwd_wgrad(c, w8 + L.h, c.f, w8 + TL.dy_perm, c.d, offsets, dw_down, c.f >= c.d, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_bwd_wgrad(c, w8 + L.x_perm, c.d, w8 + TL.dg, c.f, offsets, dw_gate, c.d >= c.f, stream, ctx);
+  if (e == cudaSuccess)
+    e = launch_bwd_wgrad(c, w8 + L.x_perm, c.d, w8 + TL.du, c.f, offsets, dw_up, c.d >= c.f, stream, ctx);
+  return cuda_status(e);
 }
 
 }  // extern "C"

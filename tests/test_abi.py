@@ -127,3 +127,62 @@ def test_noalloc_dispatch_rejects_oversize_before_launch(moe):
     small = _cfg(moe, T=64)
     assert moe.STATUS[moe.lib.moe_dispatch_noalloc(small.ref, None, None, ok, ok, ok, ok, ok, ok, ok, None,
                                                    None)] == "MOE_ERR_INVALID_ARG"
+
+
+def test_host_batches_argument_errors_before_launch(moe):
+    c = _cfg(moe, T=64, dtype="bf16")
+    P = ctypes.c_void_p
+    ok = P(256)
+    need = moe.workspace_size_host_batches(c)
+    base = moe.workspace_size(c)
+    assert need >= base + 2 * 64 * c.d * 2
+    arr = (P * 2)(ok, ok)
+    holes = (P * 2)(ok, None)
+    f = moe.lib.moe_layer_forward_host_batches
+    assert moe.STATUS[f(c.ref, -1, arr, ok, None, ok, ok, ok, arr, ok, need, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[f(c.ref, 2, None, ok, None, ok, ok, ok, arr, ok, need, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[f(c.ref, 2, arr, ok, None, ok, ok, ok, holes, ok, need, None)] == "MOE_ERR_INVALID_ARG"
+    # the layer workspace alone is not enough: the second staging slot is missing
+    assert moe.STATUS[f(c.ref, 2, arr, ok, None, ok, ok, ok, arr, ok, base, None)] == "MOE_ERR_WORKSPACE"
+    assert f(c.ref, 0, None, ok, None, ok, ok, ok, None, ok, need, None) == 0
+    assert moe.workspace_size_host_batches(_cfg(moe, E=4)) == 0
+
+
+def test_down_combine_scope_checked_before_launch(moe):
+    P = ctypes.c_void_p
+    ok = P(256)
+    f32 = _cfg(moe, T=1024, dtype="f32")
+    odd = _cfg(moe, T=1024, dtype="bf16", d=384)
+    small = _cfg(moe, T=64, dtype="bf16")  # weight-streaming size
+    for c in (f32, odd, small):
+        assert moe.STATUS[moe.lib.moe_expert_down_combine(c.ref, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None)] == \
+            "MOE_ERR_UNSUPPORTED"
+    big = _cfg(moe, T=1024, dtype="bf16", d=512)
+    need = moe.lib.moe_expert_down_combine_workspace_size(big.ref)
+    assert need >= 1024 * 512 * 4
+    st = moe.lib.moe_expert_down_combine(big.ref, ok, ok, ok, ok, ok, ok, ok, need - 1, None)
+    assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
+    st = moe.lib.moe_expert_down_combine(big.ref, ok, ok, ok, ok, None, ok, ok, need, None)
+    assert moe.STATUS[st] == "MOE_ERR_INVALID_ARG"
+
+
+def test_training_entry_points_checked_before_launch(moe):
+    P = ctypes.c_void_p
+    ok = P(256)
+    f32 = _cfg(moe, T=64, dtype="f32")
+    odd = _cfg(moe, T=64, dtype="bf16", d=384, f=512)
+    assert moe.workspace_size_train(f32) == 0 and moe.workspace_size_train(odd) == 0
+    for c in (f32, odd):
+        assert moe.STATUS[moe.lib.moe_layer_forward_train(c.ref, ok, ok, None, ok, ok, ok, ok, ok, 1 << 40,
+                                                          None)] == "MOE_ERR_UNSUPPORTED"
+        assert moe.STATUS[moe.lib.moe_layer_backward(c.ref, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok,
+                                                     1 << 40, None)] == "MOE_ERR_UNSUPPORTED"
+    c = _cfg(moe, T=64, dtype="bf16", d=256, f=512)
+    need = moe.workspace_size_train(c)
+    assert need > moe.workspace_size(c)
+    st = moe.lib.moe_layer_forward_train(c.ref, ok, ok, None, ok, ok, ok, ok, ok, need - 1, None)
+    assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
+    st = moe.lib.moe_layer_backward(c.ref, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ok, ok, ok, need - 1, None)
+    assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
+    st = moe.lib.moe_layer_backward(c.ref, ok, ok, ok, ok, ok, ok, ok, None, None, ok, ok, ok, ok, need, None)
+    assert moe.STATUS[st] == "MOE_ERR_INVALID_ARG"

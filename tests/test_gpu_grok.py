@@ -146,3 +146,47 @@ def test_grok_decode_int8_full_size(grok):
            for i, (L, g) in enumerate(outs)]
     REPORT["grok_decode_int8"] = {"calls_checked": list(calls), "weight_codes_bit_exact": True,
                                   "max_err_over_rms": [list(r) for r in res]}
+
+
+def test_grok_train_full_size(grok):
+    """Training pair at the full Grok prefill size, in the configuration the
+    benchmark times: dx on sampled tokens (each differentiated in fp64 by the
+    oracle), and for two experts whole columns of dW_gate / dW_up and rows of
+    dW_down (the oracle's hidden-unit slices), within the backward bar."""
+    import sparse_moe_layer_07_b200 as moe
+    from synth import normal
+
+    host, dev = grok
+    w = W["grok_prefill"]
+    L = LayerInputs(w, host=host, dev_weights=dev)
+    c = L.cfg
+    ws = torch.empty(moe.workspace_size_train(c), dtype=torch.uint8, device="cuda")
+    moe.layer_forward_train(c, L.dev["x"], dev["wr"], dev["wg"], dev["wu"], dev["wd"], ws)
+    go = normal(configs.SEED, 907, (w.T, w.d), dtype="bf16")
+    g = moe.layer_backward(c, L.dev["x"], dev["wr"], dev["wg"], dev["wu"], dev["wd"], to_dev(go), ws)
+    torch.cuda.synchronize()
+    assert moe.get_device_error() == 0
+    tol = 8e-2  # max |err| over RMS, the backward bar of test_gpu_train
+    tokens = _sample(w.T, 14, 13)
+    ref = oracle.layer_backward(L.x, L.wr, L.wg, L.wu, L.wd, w.capacity_factor, go, tokens=tokens)
+    gap = oracle.near_tie_gap(ref["logits"])[tokens]
+    rows = tokens[gap > 1e-3]
+    dx = g["dx"].float().cpu().numpy().astype(np.float64)[rows]
+    want = ref["dx"][rows]
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    err_dx = float(np.max(np.abs(dx - want))) / rms
+    assert err_dx <= tol, err_dx
+    res = {"dx_tokens": int(rows.size), "dx_max_err_over_rms": err_dx}
+    cols = [0, 1, 12345, w.f - 1]
+    for e in (0, 5):
+        sl = oracle.expert_weight_grad_slices(L.x, L.wr, L.wg, L.wu, L.wd, w.capacity_factor, go, e, cols)
+        pairs = (("dw_gate", g["dw_gate"][e][:, cols], sl["dw_gate_cols"]),
+                 ("dw_up", g["dw_up"][e][:, cols], sl["dw_up_cols"]),
+                 ("dw_down", g["dw_down"][e][cols, :], sl["dw_down_rows"]))
+        for name, got_t, want in pairs:
+            got = got_t.cpu().numpy().astype(np.float64)
+            rms = float(np.sqrt(np.mean(want ** 2)))
+            err = float(np.max(np.abs(got - want))) / rms
+            assert err <= tol, (name, e, err)
+            res[f"{name}_e{e}_max_err_over_rms"] = err
+    REPORT["grok_train"] = res

@@ -443,12 +443,32 @@ def pin_backward_dropped_token(o):
         np.testing.assert_allclose(r2[k], 3.0 * r[k], rtol=1e-12, atol=1e-12)
 
 
+def pin_backward_subsets_and_slices(o):
+    # the token-subset and hidden-unit-slice forms give exactly the corresponding
+    # parts of the whole backward
+    x, wr, b, wg, wu, wd, go = _bwd_case(24, T=10, d=6, f=7)
+    full = o.layer_backward(x, wr, wg, wu, wd, 1.0, go, logit_bias=b)
+    sub = [1, 4, 9]
+    part = o.layer_backward(x, wr, wg, wu, wd, 1.0, go, logit_bias=b, tokens=sub)
+    for k in ("dx", "dlogits", "dweight"):
+        np.testing.assert_allclose(part[k][sub], full[k][sub], rtol=1e-12, atol=1e-12)
+        rest = np.setdiff1d(np.arange(10), sub)
+        assert np.all(part[k][rest] == 0)
+    for e in range(8):
+        cols = [0, 3, 6]
+        sl = o.expert_weight_grad_slices(x, wr, wg, wu, wd, 1.0, go, e, cols, logit_bias=b)
+        np.testing.assert_allclose(sl["dw_gate_cols"], full["dw_gate"][e][:, cols], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sl["dw_up_cols"], full["dw_up"][e][:, cols], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sl["dw_down_rows"], full["dw_down"][e][cols, :], rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [pin_router_logits, pin_top2_brute_force, pin_softmax_closed_form, pin_zero_router,
             pin_scale_invariance, pin_capacity_values, pin_dispatch_brute_force, pin_no_drop,
             pin_hand_built_drop, pin_layer_dense_brute_force, pin_identity_experts,
             pin_two_expert_dense, pin_bf16_decoding, pin_quantize_int8,
             pin_quantized_layer_uses_dequantized_weights, pin_quantize_rows, pin_int8_layer_exact,
-            pin_backward_finite_differences, pin_backward_autograd, pin_backward_dropped_token]
+            pin_backward_finite_differences, pin_backward_autograd, pin_backward_dropped_token,
+            pin_backward_subsets_and_slices]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
