@@ -474,7 +474,7 @@ def main():
         line["decode"] = decode_bench(moe, W, dev, stream, peaks, peak_src, world)
 
     # ---- training step (forward that keeps its state + backward) on the same batch
-    if (not args.no_train and w.name == "grok_prefill" and w.storage == "bf16" and w.d % 256 == 0
+    if (not args.no_train and w.name.startswith("grok_prefill") and w.storage == "bf16" and w.d % 256 == 0
             and w.f % 256 == 0):
         line["train"] = train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, args.train_steps)
 
