@@ -148,6 +148,26 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const 
                           int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
                           void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* A batch split into token shards, one per rank, under the global capacity rule
+ * ("Routing: top-2 without auxiliary loss": capacity from the whole batch,
+ * overflow dropped lowest token index first, the shards in rank order forming
+ * the token order).  moe_route_counts writes counts[e] = assignments routed to
+ * expert e by this shard (device int32 [E]).  After every shard's counts are
+ * gathered in shard order into shard_counts [n_shards, E] (device int32; one
+ * all-gather of E integers per rank), moe_dispatch_shard computes what
+ * moe_dispatch computes for this shard with
+ *   kept iff prior[e] + rank(t, e) < capacity,  prior[e] = sum over earlier shards
+ * and counts_kept[e] = min(counts_raw[e], max(capacity - prior[e], 0)).
+ * capacity is the global one (moe_capacity of the whole batch's config);
+ * cfg->T is this shard's token count.  Deterministic, no atomics. */
+MOE_API moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                              moe_stream_t stream);
+MOE_API moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const int32_t* shard_counts,
+                                int32_t n_shards, int32_t shard, const void* x, const int32_t* topk_idx,
+                                const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
+                                int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
+                                void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* SwiGLU expert FFN over the grouped rows ("Expert implementation: SwiGLU at
  * scale", SwiGLUExpert / FusedSwiGLUExpert), for each expert e and each row r
  * in [offsets[e], offsets[e+1]):

@@ -76,6 +76,9 @@ def _load():
         "moe_workspace_size_host_batches": ([cfgp], sz),
         "moe_expert_down_combine_workspace_size": ([cfgp], sz),
         "moe_workspace_size_train": ([cfgp], sz),
+        "moe_route_counts": ([cfgp, P, P, P], ctypes.c_int),
+        "moe_dispatch_shard": ([cfgp, ctypes.c_int64, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, P, P, P,
+                                P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_train": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_layer_backward": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_expert_down_combine": ([cfgp, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
@@ -211,6 +214,45 @@ def dispatch(cfg: Config, x, topk_idx, topk_w, gather: bool = True, out=None, ws
                             _dev_ptr(o["counts_kept"]), _dev_ptr(o["offsets"]), _dev_ptr(o["perm"]),
                             _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]), _dev_ptr(o["x_perm"]),
                             _dev_ptr(ws), ws.numel(), _stream(stream, dev.device)), "moe_dispatch")
+    return o
+
+
+def route_counts(cfg: Config, topk_idx, counts=None, stream=None):
+    """counts[e] = assignments routed to expert e (device int32 [E])."""
+    if counts is None:
+        counts = _empty((cfg.E,), torch.int32, topk_idx)
+    _check(lib.moe_route_counts(cfg.ref, _dev_ptr(topk_idx), _dev_ptr(counts), _stream(stream, topk_idx.device)),
+           "moe_route_counts")
+    return counts
+
+
+def dispatch_shard(cfg: Config, capacity: int, shard_counts, shard: int, x, topk_idx, topk_w, gather: bool = True,
+                   out=None, ws=None, stream=None):
+    """Dispatch of token shard `shard` of a larger batch under the global capacity:
+    shard_counts [n_shards, E] holds every shard's route_counts in shard order.
+    Returns the same dict as dispatch()."""
+    dev = topk_idx
+    rows = cfg.T * cfg.top_k
+    o = dict(out or {})
+    o.setdefault("counts_raw", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("counts_kept", _empty((cfg.E,), torch.int32, dev))
+    o.setdefault("offsets", _empty((cfg.E + 1,), torch.int32, dev))
+    o.setdefault("perm", _empty((rows,), torch.int32, dev))
+    o.setdefault("slot_of", _empty((cfg.T, cfg.top_k), torch.int32, dev))
+    o.setdefault("row_scale", _empty((rows,), torch.float32, dev))
+    if gather:
+        o.setdefault("x_perm", _empty((rows, cfg.d), cfg.torch_dtype, dev))
+    else:
+        o["x_perm"] = None
+    if ws is None:
+        ws = _empty((max(dispatch_workspace_size(cfg), 1),), torch.uint8, dev)
+    if shard_counts.dtype != torch.int32 or shard_counts.dim() != 2 or shard_counts.shape[1] != cfg.E:
+        raise ValueError("shard_counts must be int32 [n_shards, E]")
+    _check(lib.moe_dispatch_shard(cfg.ref, int(capacity), _dev_ptr(shard_counts), shard_counts.shape[0], int(shard),
+                                  _dev_ptr(x), _dev_ptr(topk_idx), _dev_ptr(topk_w), _dev_ptr(o["counts_raw"]),
+                                  _dev_ptr(o["counts_kept"]), _dev_ptr(o["offsets"]), _dev_ptr(o["perm"]),
+                                  _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]), _dev_ptr(o["x_perm"]),
+                                  _dev_ptr(ws), ws.numel(), _stream(stream, dev.device)), "moe_dispatch_shard")
     return o
 
 

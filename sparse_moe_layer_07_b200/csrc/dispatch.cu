@@ -8,6 +8,11 @@
 // lowest-token-index-first, i.e. assignment (t, e) is kept iff fewer than
 // `cap` tokens before t were routed to e.
 //
+// A batch split into token shards (one per rank) keeps the global rule: shard i
+// is told how many assignments each expert received from shards 0..i-1 and
+// keeps (t, e) iff that prior count plus t's rank inside the shard is below the
+// global capacity.
+//
 // Three deterministic passes, no atomics on any output:
 //   hist : block b counts its tokens' assignments per expert   -> block_hist[b][e]
 //   scan : exclusive scan over blocks per expert, counts, caps, offsets
@@ -60,8 +65,19 @@ __global__ void __launch_bounds__(kBT) dispatch_hist_kernel(const int32_t* __res
   }
 }
 
+// Assignments routed to each expert by the tokens of earlier shards (the first
+// `shard` rows of shard_counts [n_shards, E]), 0 without shards.
+__device__ __forceinline__ int64_t prior_count(const int32_t* shard_counts, int shard, int e) {
+  int64_t p = 0;
+  if (shard_counts)
+    for (int r = 0; r < shard; ++r) p += shard_counts[r * kE + e];
+  return p;
+}
+
 // One block of 8 warps; warp e scans block_hist[:, e] in chunks of 32 blocks.
+// With shards, expert e has cap - prior slots left for this shard's tokens.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict__ block_hist, int64_t nblk, int64_t cap,
+                                                           const int32_t* __restrict__ shard_counts, int shard,
                                                            int32_t* __restrict__ counts_raw,
                                                            int32_t* __restrict__ counts_kept,
                                                            int32_t* __restrict__ offsets, int32_t* __restrict__ stats) {
@@ -86,7 +102,9 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
     int off = 0, dropped = 0;
     for (int k = 0; k < kE; ++k) {
       const int raw = s_total[k];
-      const int kept = (int64_t)raw < cap ? raw : (int)cap;
+      int64_t left = cap - prior_count(shard_counts, shard, k);
+      if (left < 0) left = 0;
+      const int kept = (int64_t)raw < left ? raw : (int)left;
       counts_raw[k] = raw;
       counts_kept[k] = kept;
       offsets[k] = off;
@@ -108,6 +126,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
 
 __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
                                                            int64_t T, int64_t cap,
+                                                           const int32_t* __restrict__ shard_counts, int shard,
                                                            const int32_t* __restrict__ block_base,
                                                            const int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ perm, int32_t* __restrict__ slot_of,
@@ -115,6 +134,7 @@ __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __res
   __shared__ int s_cnt[kWarps][kE];
   __shared__ int s_base[kE];
   __shared__ int s_off[kE];
+  __shared__ int64_t s_prior[kE];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * kBT + threadIdx.x;
   int e0, e1;
@@ -122,6 +142,7 @@ __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __res
   if (threadIdx.x < kE) {
     s_base[threadIdx.x] = block_base[(int64_t)blockIdx.x * kE + threadIdx.x];
     s_off[threadIdx.x] = offsets[threadIdx.x];
+    s_prior[threadIdx.x] = prior_count(shard_counts, shard, threadIdx.x);
   }
   const unsigned lt = (1u << lane) - 1u;
   int pre0 = 0, pre1 = 0;  // in-warp prefix for this lane's slot 0 / slot 1
@@ -147,7 +168,7 @@ __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __res
     if (e < 0) continue;
     int r = s_base[e] + pres[j];
     for (int k = 0; k < warp; ++k) r += s_cnt[k][e];
-    if ((int64_t)r < cap) {
+    if (s_prior[e] + r < cap) {
       const int s = s_off[e] + r;
       slots[j] = s;
       perm[s] = (int32_t)t;
@@ -194,16 +215,50 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 cudaError_t launch_dispatch(const moe_config_t& c, int64_t cap, const int32_t* idx, const float* w,
                             int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets,
                             int32_t* perm, int32_t* slot_of, float* row_scale, int32_t* block_hist,
-                            int32_t* stats, cudaStream_t s, const Ctx& ctx) {
+                            int32_t* stats, cudaStream_t s, const Ctx& ctx, const int32_t* shard_counts,
+                            int shard) {
   const int64_t nblk = dispatch_blocks(c);
   if (nblk > 0) {
     dispatch_hist_kernel<<<(unsigned)nblk, kBT, 0, s>>>(idx, c.T, block_hist, ctx.err);
   }
-  dispatch_scan_kernel<<<1, 256, 0, s>>>(block_hist, nblk, cap, counts_raw, counts_kept, offsets, stats);
+  dispatch_scan_kernel<<<1, 256, 0, s>>>(block_hist, nblk, cap, shard_counts, shard, counts_raw, counts_kept,
+                                          offsets, stats);
   if (nblk > 0) {
-    dispatch_rank_kernel<<<(unsigned)nblk, kBT, 0, s>>>(idx, w, c.T, cap, block_hist, offsets, perm, slot_of,
-                                                        row_scale, ctx.err);
+    dispatch_rank_kernel<<<(unsigned)nblk, kBT, 0, s>>>(idx, w, c.T, cap, shard_counts, shard, block_hist, offsets,
+                                                        perm, slot_of, row_scale, ctx.err);
   }
+  return cudaGetLastError();
+}
+
+// counts[e] = assignments routed to e over the whole batch: one block, each
+// thread counts a strided share of the tokens, then a fixed-order reduction.
+__global__ void __launch_bounds__(256) route_counts_kernel(const int32_t* __restrict__ idx, int64_t T,
+                                                          int32_t* __restrict__ counts, int* err) {
+  __shared__ int s[kE][256];
+  int c[kE];
+#pragma unroll
+  for (int e = 0; e < kE; ++e) c[e] = 0;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+    int e0, e1;
+    load_pair(idx, t, T, e0, e1, err);
+#pragma unroll
+    for (int e = 0; e < kE; ++e) c[e] += (e0 == e) + (e1 == e);
+  }
+#pragma unroll
+  for (int e = 0; e < kE; ++e) s[e][threadIdx.x] = c[e];
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w)
+#pragma unroll
+      for (int e = 0; e < kE; ++e) s[e][threadIdx.x] += s[e][threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x < kE) counts[threadIdx.x] = s[threadIdx.x][0];
+}
+
+cudaError_t launch_route_counts(const moe_config_t& c, const int32_t* idx, int32_t* counts, cudaStream_t s,
+                                const Ctx& ctx) {
+  route_counts_kernel<<<1, 256, 0, s>>>(idx, c.T, counts, ctx.err);
   return cudaGetLastError();
 }
 

@@ -16,8 +16,9 @@
 //         two terms per token, so the order of the adds does not matter)
 //   kWG : dW[e] = A_e^T B_e over the rows of expert e  (A, B MN-major:
 //         dW_down = H^T (w * dout),  dW_gate = X^T dG,  dW_up = X^T dU); K is
-//         the ragged row count, the rows past the expert's end in its last K
-//         block are zeroed in shared memory before the MMA.
+//         the ragged row count: the expert's last K block issues only the
+//         16-row MMA steps that hold its rows, and the rows of the last step
+//         past the expert's end are zeroed in shared memory before the MMA.
 // Pipeline as in ffn_tc.cu: persistent CTAs, warp 0 TMA, warp 1 MMA + TMEM
 // (two 128 x 256 fp32 accumulators), warps 2-5 epilogue; every wait bounded.
 #include <cuda.h>
@@ -44,7 +45,11 @@ constexpr int A_BYTES = 2 * CHUNK;      // 16 KB: 128 x 64
 constexpr int B_BYTES = 4 * CHUNK;      // 32 KB: 256 x 64
 constexpr int STAGE = A_BYTES + B_BYTES;
 constexpr int kStages = 4;
-constexpr int SMEM_BYTES = 1024 + kStages * STAGE + 256;
+// weight gradients: each epilogue warp stages 32 rows x 32 fp32 (4 KB, 128-byte
+// swizzled) for a TMA tile store, double buffered
+constexpr int OUT_STAGE = 32 * 32 * 4;
+constexpr int OUT_BYTES = 4 * 2 * OUT_STAGE;
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE + OUT_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 enum Mode { kDH = 0, kDX = 1, kWG = 2 };
@@ -161,14 +166,15 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                    const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tmOut, const BwdArgs args) {
   constexpr int S = kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * STAGE);
+  uint8_t* sOut = smem + S * STAGE;  // 1024-byte aligned: S * STAGE is a multiple of 1024
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * STAGE + OUT_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -289,20 +295,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        // K steps of 16 rows issued for this block: the expert's last block issues
+        // only the steps that hold its rows, and the rows of the last such step
+        // past the expert's end (next expert's rows, or past the kept rows) are
+        // zeroed in both operands first (each row is 128 bytes of every chunk).
+        int ksteps = BK / 16;
         if (MODE == kWG) {
           const int valid = t.nrows - kb * BK;
           if (valid < BK) {
-            // rows [valid, 64) of the 6 chunks (2 of A, 4 of B) belong to the next
-            // expert or lie past the kept rows: zero them (each row is 128 bytes)
-            uint8_t* base = sA + s * A_BYTES;
-            const int per_chunk = (BK - valid) * 8;  // 16-byte pieces
-            for (int i = lane; i < 6 * per_chunk; i += 32) {
-              const int c = i / per_chunk;
-              const int j = i - c * per_chunk;
-              uint8_t* chunk = c < 2 ? base + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
-              *reinterpret_cast<uint4*>(chunk + valid * 128 + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+            ksteps = (valid + 15) / 16;
+            const int pad = ksteps * 16 - valid;
+            if (pad > 0) {
+              const int per_chunk = pad * 8;  // 16-byte pieces
+              for (int i = lane; i < 6 * per_chunk; i += 32) {
+                const int c = i / per_chunk;
+                const int j = i - c * per_chunk;
+                uint8_t* chunk = c < 2 ? sA + s * A_BYTES + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
+                *reinterpret_cast<uint4*>(chunk + valid * 128 + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             __syncwarp();
           }
         }
@@ -312,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
+            if (kk >= ksteps) break;
             uint64_t ad, bd;
             if (kMN) {
               ad = sw128_desc(a_addr + kk * 2048, CHUNK, 1024);
@@ -423,19 +436,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        float* dst = args.out + ((int64_t)t.e * args.M + t.m0 + r) * args.ld + t.n0;
+        // 32 rows x 32 columns per TMA store: lane = row, its 8 16-byte pieces
+        // placed with the 128-byte swizzle (piece j of row r at j ^ (r % 8))
         const bool zero = t.nkb == 0;
+        uint8_t* stage0 = sOut + (q * 2) * OUT_STAGE;
+        const int y = t.e * (int)args.M + t.m0 + q * 32;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
           tmem_wait_ld();
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+          uint8_t* st = stage0 + (c & 1) * OUT_STAGE;
+          if (lane == 0) bulk_wait_group_read<1>();  // the store that last read this buffer is done with it
+          __syncwarp();
+          float4* row = reinterpret_cast<float4*>(st + lane * 128);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                         : make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          for (int j = 0; j < 8; ++j)
+            row[j ^ (lane & 7)] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                       : make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, st, t.n0 + c * 32, y);
+            bulk_commit_group();
+          }
         }
       }
       tc_fence_before();
@@ -443,6 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // tile stores still in flight must finish before the CTA (and its shared memory) goes
+  if (MODE == kWG && warp >= 2 && lane == 0) bulk_wait_group_all();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -452,11 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int MODE>
 cudaError_t launch_bwd(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const BwdArgs& args, cudaStream_t s, const Ctx& ctx) {
+                       const CUtensorMap& out, const BwdArgs& args, cudaStream_t s, const Ctx& ctx) {
   auto kern = bwd_gemm_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<ctx.num_sms, kThreads, SMEM_BYTES, s>>>(a0, a1, b0, b1, args);
+  kern<<<ctx.num_sms, kThreads, SMEM_BYTES, s>>>(a0, a1, b0, b1, out, args);
   return cudaGetLastError();
 }
 
@@ -506,7 +533,7 @@ cudaError_t launch_bwd_dh(const moe_config_t& c, const void* dout_perm, const in
   a.dU = static_cast<__nv_bfloat16*>(dU);
   a.dw_part = dw_part;
   a.ld = c.f;
-  return launch_bwd<kDH>(ta, ta, tb, tb, a, s, ctx);
+  return launch_bwd<kDH>(ta, ta, tb, tb, ta, a, s, ctx);
 }
 
 cudaError_t launch_bwd_dx(const moe_config_t& c, const void* dG, const void* dU, const int32_t* offsets,
@@ -526,15 +553,21 @@ cudaError_t launch_bwd_dx(const moe_config_t& c, const void* dG, const void* dU,
   a.perm = perm;
   a.out = dx32;
   a.ld = c.d;
-  return launch_bwd<kDX>(ta0, ta1, tb0, tb1, a, s, ctx);
+  return launch_bwd<kDX>(ta0, ta1, tb0, tb1, ta0, a, s, ctx);
 }
 
 cudaError_t launch_bwd_wgrad(const moe_config_t& c, const void* a_rows, int64_t M, const void* b_rows, int64_t N,
                              const int32_t* offsets, float* dW, bool m_outer, cudaStream_t s, const Ctx& ctx) {
   const int64_t rows = slot_rows(c);
   if (rows == 0 || M % BM != 0 || N % BN != 0) return rows == 0 ? cudaSuccess : cudaErrorInvalidValue;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to;
   if (!map_rows(&ta, a_rows, rows, M, 64) || !map_rows(&tb, b_rows, rows, N, 64)) return cudaErrorInvalidValue;
+  // dW [E * M, N] fp32, stored 32 x 32 at a time from the swizzled staging tiles
+  const uint64_t o_dims[2] = {(uint64_t)N, (uint64_t)c.E * M};
+  const uint64_t o_str[1] = {(uint64_t)N * 4};
+  const uint32_t o_box[2] = {32, 32};
+  if (!encode_tmap_dtype(&to, dW, 2, o_dims, o_str, o_box, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+    return cudaErrorInvalidValue;
   BwdArgs a = base_args(c, offsets, ctx);
   a.m_tiles = (int)(M / BM);
   a.n_tiles = (int)(N / BN);
@@ -542,7 +575,7 @@ cudaError_t launch_bwd_wgrad(const moe_config_t& c, const void* a_rows, int64_t 
   a.out = dW;
   a.ld = N;
   a.M = M;
-  return launch_bwd<kWG>(ta, ta, tb, tb, a, s, ctx);
+  return launch_bwd<kWG>(ta, ta, tb, tb, to, a, s, ctx);
 }
 
 }  // namespace moe

@@ -31,7 +31,11 @@ cudaError_t launch_router(const moe_config_t& c, const void* x, const void* wr, 
 cudaError_t launch_dispatch(const moe_config_t& c, int64_t cap, const int32_t* idx, const float* w,
                             int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets,
                             int32_t* perm, int32_t* slot_of, float* row_scale, int32_t* block_hist,
-                            int32_t* stats, cudaStream_t s, const Ctx& ctx);
+                            int32_t* stats, cudaStream_t s, const Ctx& ctx,
+                            const int32_t* shard_counts = nullptr, int shard = 0);
+// counts[e] = number of assignments routed to expert e (one block, fixed order).
+cudaError_t launch_route_counts(const moe_config_t& c, const int32_t* idx, int32_t* counts, cudaStream_t s,
+                                const Ctx& ctx);
 
 cudaError_t launch_gather(const moe_config_t& c, const void* x, const int32_t* perm,
                           const int32_t* offsets, void* x_perm, cudaStream_t s, const Ctx& ctx);

@@ -258,6 +258,40 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   return cuda_status(e);
 }
 
+moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                              moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || (cfg->T > 0 && (!topk_idx || !aligned16(topk_idx)))) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  return cuda_status(launch_route_counts(*cfg, topk_idx, counts, stream, ctx));
+}
+
+moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const int32_t* shard_counts,
+                                int32_t n_shards, int32_t shard, const void* x, const int32_t* topk_idx,
+                                const float* topk_w, int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets,
+                                int32_t* perm, int32_t* slot_of, float* row_scale, void* x_perm, void* ws,
+                                size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (capacity < 0 || n_shards < 1 || shard < 0 || shard >= n_shards || !shard_counts) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx || !topk_w || !counts_raw || !counts_kept || !offsets || !perm || !slot_of || !row_scale)
+    return MOE_ERR_INVALID_ARG;
+  if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(slot_of) || (x_perm && !aligned16(x_perm)) ||
+      (x && !aligned16(x)))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < dispatch_ws(*cfg) || (dispatch_ws(*cfg) > 0 && !ws)) return MOE_ERR_WORKSPACE;
+  Ctx ctx;
+  if ((st = get_ctx(ctx)) != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  cudaError_t e = launch_dispatch(c, capacity, topk_idx, topk_w, counts_raw, counts_kept, offsets, perm, slot_of,
+                                  row_scale, static_cast<int32_t*>(ws), nullptr, stream, ctx, shard_counts, shard);
+  if (e == cudaSuccess && x_perm && c.T > 0) e = launch_gather(c, x, perm, offsets, x_perm, stream, ctx);
+  return cuda_status(e);
+}
+
 moe_status_t moe_expert_gate_up(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
                                 const void* w_gate, const void* w_up, void* h, moe_stream_t stream) {
   moe_status_t st = check_config(cfg);

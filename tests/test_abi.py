@@ -186,3 +186,20 @@ def test_training_entry_points_checked_before_launch(moe):
     assert moe.STATUS[st] == "MOE_ERR_WORKSPACE"
     st = moe.lib.moe_layer_backward(c.ref, ok, ok, ok, ok, ok, ok, ok, None, None, ok, ok, ok, ok, need, None)
     assert moe.STATUS[st] == "MOE_ERR_INVALID_ARG"
+
+
+def test_shard_dispatch_arguments_checked_before_launch(moe):
+    P = ctypes.c_void_p
+    ok = P(256)
+    c = _cfg(moe, T=64)
+    ws = moe.dispatch_workspace_size(c)
+    f = moe.lib.moe_dispatch_shard
+    assert moe.STATUS[f(c.ref, 10, ok, 2, 2, None, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws, None)] == \
+        "MOE_ERR_INVALID_ARG"  # shard index out of range
+    assert moe.STATUS[f(c.ref, -1, ok, 2, 0, None, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws, None)] == \
+        "MOE_ERR_INVALID_ARG"  # negative capacity
+    assert moe.STATUS[f(c.ref, 10, None, 2, 0, None, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws, None)] == \
+        "MOE_ERR_INVALID_ARG"  # no count table
+    assert moe.STATUS[f(c.ref, 10, ok, 2, 0, None, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws - 1, None)] == \
+        "MOE_ERR_WORKSPACE"
+    assert moe.STATUS[moe.lib.moe_route_counts(c.ref, ok, None, None)] == "MOE_ERR_INVALID_ARG"

@@ -65,3 +65,67 @@ def test_two_gloo_ranks():
     assert not np.array_equal(res[0][2], res[1][2])
     assert res[0][3] == res[1][3] == 5.0
     assert res[0][4] == pytest.approx(2 * 16 * 10 / 0.005)
+
+
+def _shard_worker(rank, world, port, q):
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import oracle
+    from sparse_moe_layer_07_b200.sharded import gather_shard_counts
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        idx, _, cap, per = _global_routing(oracle)
+        mine = idx[rank * per:(rank + 1) * per]
+        counts = torch.from_numpy(np.bincount(mine.ravel(), minlength=8).astype(np.int32))
+        table = gather_shard_counts(counts).numpy()
+        prior = table[:rank].sum(0)
+        seen = np.zeros(8, dtype=np.int64)
+        kept = np.zeros(mine.shape, dtype=bool)
+        for t in range(per):
+            for j in range(2):
+                e = mine[t, j]
+                kept[t, j] = prior[e] + seen[e] < cap
+                seen[e] += 1
+        q.put((rank, table, kept))
+    finally:
+        dist.destroy_process_group()
+
+
+def _global_routing(oracle):
+    rng = np.random.default_rng(31)
+    T, d = 90, 16
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((8, d)) * 0.3
+    lg = oracle.router_logits(x, wr, np.array([1.5, 0.5, 0, 0, 0, 0, 0, 0]))
+    idx, w = oracle.top2_softmax(lg)
+    return idx, w, oracle.capacity(T, 2, 8, 1.0), T // 3
+
+
+def test_three_gloo_ranks_shard_the_global_capacity():
+    # each rank holds a contiguous third of the batch; one all-gather of the E route
+    # counts per rank lets every rank apply the global lowest-index-first rule alone
+    import oracle
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(3):
+        r = q.get(timeout=120)
+        res[r[0]] = r
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    idx, w, cap, per = _global_routing(oracle)
+    ref = oracle.dispatch(idx, w, 8, cap)
+    assert ref["dropped"] > 0
+    want_table = np.stack([np.bincount(idx[r * per:(r + 1) * per].ravel(), minlength=8) for r in range(3)])
+    for r in range(3):
+        assert np.array_equal(res[r][1], want_table)
+    kept = np.concatenate([res[r][2] for r in range(3)])
+    assert np.array_equal(kept, ref["slot_of"] >= 0)
