@@ -8,8 +8,9 @@
 // with G = X W_gate, U = X W_up, H = silu(G) * U saved by the forward:
 //   kDH : dHu[r, :] = dout[t, :] W_down[e]^T        (A = dout rows, B = W_down K-major)
 //         epilogue: dH = w * dHu,  dG = dH * U * silu'(G),  dU = dH * silu(G),
-//         and a per-tile partial of <dHu, H> (= the routing weight's gradient
-//         <dout, y>), summed later in a fixed order
+//         and per-tile partials of <dHu, H> (= the routing weight's gradient
+//         <dout, y>; two per tile, one per half of its columns), summed later
+//         in a fixed order
 //   kDX : dx[t, :] += dG[r, :] W_gate[e]^T + dU[r, :] W_up[e]^T
 //         (K runs over both halves; B = W_gate / W_up read K-major straight from
 //         their [E, d, f] layout; the epilogue adds into an fp32 sum by token:
@@ -37,7 +38,14 @@ constexpr int kE = 8;
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+// Epilogue warps: 4 (one per TMEM lane quarter), or 8 for kDH, whose epilogue
+// reads G, U, H and writes dG, dU for every element: there the two warps of a
+// lane quarter take half of the tile's columns each, doubling the loads in flight.
+template <int MODE>
+struct Warps {
+  static constexpr int kEpi = MODE == 0 ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpi;
+};
 constexpr int kTmemCols = 512;
 constexpr int kAccStride = 256;
 constexpr int CHUNK = 64 * BK * 2;      // 8 KB: 64 x 64 bf16
@@ -70,7 +78,7 @@ struct BwdArgs {
   const __nv_bfloat16* H;
   __nv_bfloat16* dG;       // kDH outputs [rows, f]
   __nv_bfloat16* dU;
-  float* dw_part;          // kDH: [rows, n_tiles]
+  float* dw_part;          // kDH: [rows, 2 * n_tiles] (two column halves per tile)
   float* out;              // kDX: dx32 [T, d];  kWG: dW [E, M, N]
   int64_t ld;              // kDH: f;  kDX: d;  kWG: N
   int64_t M;               // kWG
@@ -163,7 +171,7 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmOut, const BwdArgs args) {
@@ -193,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], 32 * Warps<MODE>::kEpi);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -357,6 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    // column chunks of 32 this warp covers: all 8, or one half with 8 epilogue warps
+    constexpr int kSplit = Warps<MODE>::kEpi / 4;
+    const int half = kSplit == 1 ? 0 : (warp - 2) / 4;
+    const int c_begin = half * (BN / 32) / kSplit, c_end = c_begin + (BN / 32) / kSplit;
     uint32_t tc = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
       const Tile t = decode_tile<MODE>(sched, args, L);
@@ -376,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t base = row * args.ld + t.n0;
         float dot = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = c_begin; c < c_end; ++c) {
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
           tmem_wait_ld();
@@ -411,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (valid) args.dw_part[row * args.n_tiles + t.nb] = dot;
+        if (valid) args.dw_part[row * (int64_t)args.n_tiles * kSplit + t.nb * kSplit + half] = dot;
       } else if (MODE == kDX) {
         int tok = -1;
         if (r < t.rows) {
@@ -483,7 +495,7 @@ cudaError_t launch_bwd(const CUtensorMap& a0, const CUtensorMap& a1, const CUten
   auto kern = bwd_gemm_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<ctx.num_sms, kThreads, SMEM_BYTES, s>>>(a0, a1, b0, b1, out, args);
+  kern<<<ctx.num_sms, Warps<MODE>::kThreads, SMEM_BYTES, s>>>(a0, a1, b0, b1, out, args);
   return cudaGetLastError();
 }
 

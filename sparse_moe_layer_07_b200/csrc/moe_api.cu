@@ -713,7 +713,7 @@ TrainLayout train_layout_of(const moe_config_t& c) {
   L.dy_perm = take(rows * c.d * 2);
   L.dg = take(rows * c.f * 2);
   L.du = take(rows * c.f * 2);
-  L.dw_part = take(rows * (size_t)(c.f / 256) * 4);
+  L.dw_part = take(rows * (size_t)(c.f / 256) * 2 * 4);
   L.dlogits = take((size_t)c.T * c.E * 4);
   L.dweight = take((size_t)c.T * c.top_k * 4);
   L.dx32 = take((size_t)c.T * c.d * 4);
@@ -809,7 +809,7 @@ moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const vo
   const float* row_scale = reinterpret_cast<const float*>(w8 + L.row_scale);
   float* dw_part = reinterpret_cast<float*>(w8 + TL.dw_part);
   float* dx32 = reinterpret_cast<float*>(w8 + TL.dx32);
-  const int n_parts = (int)(c.f / 256);
+  const int n_parts = (int)(c.f / 256) * 2;  // two column halves per dH tile
   cudaError_t e = launch_bwd_gather(c, dout, perm, offsets, row_scale, w8 + TL.dout_perm, w8 + TL.dy_perm, stream, ctx);
   if (e == cudaSuccess)
     e = launch_bwd_dh(c, w8 + TL.dout_perm, offsets, w_down, w8 + TL.g, w8 + TL.u, w8 + L.h, row_scale, w8 + TL.dg,

@@ -24,7 +24,7 @@ CASES = {
     # skewed router, cf 1.0: expert 0 overflows, so later shards lose assignments
     "shard_skew_drop": (W["grok_skew"], dict(T=1000, d=256, f=384, capacity_factor=1.0), (300, 400, 300)),
     # every shard above the weight-streaming size, so shards and batch run the same kernels
-    "shard_uneven": (W["mid_bf16"], dict(T=1100, d=256, f=256, capacity_factor=1.1), (257, 586, 257)),
+    "shard_uneven": (W["mid_bf16"], dict(T=1100, d=256, f=256, capacity_factor=0.9), (257, 586, 257)),
     "shard_fp32": (W["tiny_f32"], dict(T=640, d=128, f=192, capacity_factor=1.0), (200, 440)),
 }
 
