@@ -160,6 +160,15 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const 
  * and counts_kept[e] = min(counts_raw[e], max(capacity - prior[e], 0)).
  * capacity is the global one (moe_capacity of the whole batch's config);
  * cfg->T is this shard's token count.  Deterministic, no atomics. */
+/* Row gather, dst[i, :] = src[idx[i], :] for i < n: rows of row_bytes bytes
+ * (a multiple of 16), src holding n_src rows (device memory; idx device int32).
+ * Used to regroup rows between the expert-major order of a rank's own experts
+ * and the rank-major order of an all-to-all exchange (expert parallelism,
+ * "Expert parallelism vs. tensor parallelism", moe_layer_ep_forward).  An
+ * index outside [0, n_src) skips its row and sets MOE_DEVERR_SLOT_INDEX. */
+MOE_API moe_status_t moe_gather_rows(const void* src, int64_t n_src, const int32_t* idx, int64_t n,
+                             int64_t row_bytes, void* dst, moe_stream_t stream);
+
 MOE_API moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
                               moe_stream_t stream);
 MOE_API moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const int32_t* shard_counts,

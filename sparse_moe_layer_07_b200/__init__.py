@@ -77,6 +77,7 @@ def _load():
         "moe_expert_down_combine_workspace_size": ([cfgp], sz),
         "moe_workspace_size_train": ([cfgp], sz),
         "moe_route_counts": ([cfgp, P, P, P], ctypes.c_int),
+        "moe_gather_rows": ([P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int64, P, P], ctypes.c_int),
         "moe_dispatch_shard": ([cfgp, ctypes.c_int64, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, P, P, P,
                                 P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_train": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
@@ -215,6 +216,19 @@ def dispatch(cfg: Config, x, topk_idx, topk_w, gather: bool = True, out=None, ws
                             _dev_ptr(o["slot_of"]), _dev_ptr(o["row_scale"]), _dev_ptr(o["x_perm"]),
                             _dev_ptr(ws), ws.numel(), _stream(stream, dev.device)), "moe_dispatch")
     return o
+
+
+def gather_rows(src, idx, out=None, stream=None):
+    """out[i] = src[idx[i]] along dim 0 (moe_gather_rows); rows of a multiple of 16 bytes."""
+    n = idx.numel()
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else src.stride(0) * src.element_size()
+    if out is None:
+        out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    if idx.dtype != torch.int32:
+        raise ValueError("idx must be int32")
+    _check(lib.moe_gather_rows(_dev_ptr(src), src.shape[0], _dev_ptr(idx), n, row_bytes, _dev_ptr(out),
+                               _stream(stream, src.device)), "moe_gather_rows")
+    return out
 
 
 def route_counts(cfg: Config, topk_idx, counts=None, stream=None):

@@ -230,6 +230,8 @@ cudaError_t launch_dispatch(const moe_config_t& c, int64_t cap, const int32_t* i
   return cudaGetLastError();
 }
 
+namespace {
+
 // counts[e] = assignments routed to e over the whole batch: one block, each
 // thread counts a strided share of the tokens, then a fixed-order reduction.
 __global__ void __launch_bounds__(256) route_counts_kernel(const int32_t* __restrict__ idx, int64_t T,
@@ -256,9 +258,44 @@ __global__ void __launch_bounds__(256) route_counts_kernel(const int32_t* __rest
   if (threadIdx.x < kE) counts[threadIdx.x] = s[threadIdx.x][0];
 }
 
+}  // namespace
+
 cudaError_t launch_route_counts(const moe_config_t& c, const int32_t* idx, int32_t* counts, cudaStream_t s,
                                 const Ctx& ctx) {
   route_counts_kernel<<<1, 256, 0, s>>>(idx, c.T, counts, ctx.err);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// dst[i] = src[idx[i]] for i < n (rows of row_vec 16-byte vectors); an index
+// outside [0, n_src) leaves its row untouched and sets the error word.
+__global__ void __launch_bounds__(256) gather_index_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ idx,
+                                                          int64_t n, int64_t n_src, int64_t row_vec,
+                                                          uint4* __restrict__ dst, int* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = gw; i < n; i += nw) {
+    const int32_t r = __ldg(idx + i);
+    if (r < 0 || r >= n_src) {
+      if (lane == 0) flag_error(err, MOE_DEVERR_SLOT_INDEX);
+      continue;
+    }
+    for (int64_t v = lane; v < row_vec; v += 32) dst[i * row_vec + v] = __ldg(src + (int64_t)r * row_vec + v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gather_index(const void* src, const int32_t* idx, int64_t n, int64_t n_src, int64_t row_bytes,
+                                void* dst, cudaStream_t s, const Ctx& ctx) {
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 7) / 8;
+  const int64_t cap_blocks = (int64_t)ctx.num_sms * 8;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  gather_index_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(src), idx, n, n_src, row_bytes / 16,
+                                                       static_cast<uint4*>(dst), ctx.err);
   return cudaGetLastError();
 }
 

@@ -9,8 +9,7 @@
 //   kDH : dHu[r, :] = dout[t, :] W_down[e]^T        (A = dout rows, B = W_down K-major)
 //         epilogue: dH = w * dHu,  dG = dH * U * silu'(G),  dU = dH * silu(G),
 //         and per-tile partials of <dHu, H> (= the routing weight's gradient
-//         <dout, y>; two per tile, one per half of its columns), summed later
-//         in a fixed order
+//         <dout, y>), summed later in a fixed order
 //   kDX : dx[t, :] += dG[r, :] W_gate[e]^T + dU[r, :] W_up[e]^T
 //         (K runs over both halves; B = W_gate / W_up read K-major straight from
 //         their [E, d, f] layout; the epilogue adds into an fp32 sum by token:
@@ -38,12 +37,12 @@ constexpr int kE = 8;
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-// Epilogue warps: 4 (one per TMEM lane quarter), or 8 for kDH, whose epilogue
-// reads G, U, H and writes dG, dU for every element: there the two warps of a
-// lane quarter take half of the tile's columns each, doubling the loads in flight.
+// Epilogue warps: 4, one per TMEM lane quarter.  (The layout also allows 8, two
+// per quarter each taking half of the tile's columns; for kDH that measured 14%
+// slower than 4 relative to the forward GEMMs in the same capture.)
 template <int MODE>
 struct Warps {
-  static constexpr int kEpi = MODE == 0 ? 8 : 4;
+  static constexpr int kEpi = 4;
   static constexpr int kThreads = 64 + 32 * kEpi;
 };
 constexpr int kTmemCols = 512;
@@ -78,7 +77,7 @@ struct BwdArgs {
   const __nv_bfloat16* H;
   __nv_bfloat16* dG;       // kDH outputs [rows, f]
   __nv_bfloat16* dU;
-  float* dw_part;          // kDH: [rows, 2 * n_tiles] (two column halves per tile)
+  float* dw_part;          // kDH: [rows, n_tiles * parts per tile]
   float* out;              // kDX: dx32 [T, d];  kWG: dW [E, M, N]
   int64_t ld;              // kDH: f;  kDX: d;  kWG: N
   int64_t M;               // kWG
@@ -524,6 +523,8 @@ bool map_weights(CUtensorMap* m, const void* base, int E, int64_t R, int64_t C) 
 }
 
 }  // namespace
+
+int bwd_dh_parts_per_tile() { return Warps<kDH>::kEpi / 4; }
 
 cudaError_t launch_bwd_dh(const moe_config_t& c, const void* dout_perm, const int32_t* offsets, const void* wd,
                           const void* G, const void* U, const void* H, const float* row_scale, void* dG, void* dU,

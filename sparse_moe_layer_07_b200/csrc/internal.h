@@ -33,6 +33,9 @@ cudaError_t launch_dispatch(const moe_config_t& c, int64_t cap, const int32_t* i
                             int32_t* perm, int32_t* slot_of, float* row_scale, int32_t* block_hist,
                             int32_t* stats, cudaStream_t s, const Ctx& ctx,
                             const int32_t* shard_counts = nullptr, int shard = 0);
+// dst[i] = src[idx[i]], i < n: rows of row_bytes (a multiple of 16) from a source of n_src rows.
+cudaError_t launch_gather_index(const void* src, const int32_t* idx, int64_t n, int64_t n_src, int64_t row_bytes,
+                                void* dst, cudaStream_t s, const Ctx& ctx);
 // counts[e] = number of assignments routed to expert e (one block, fixed order).
 cudaError_t launch_route_counts(const moe_config_t& c, const int32_t* idx, int32_t* counts, cudaStream_t s,
                                 const Ctx& ctx);
@@ -69,6 +72,8 @@ cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const i
 // Backward of the expert FFNs (bf16, d and f multiples of 256): dG / dU and the
 // routing-weight partials, dx (added into a zeroed fp32 dx32 by token), and
 // the weight gradients dW[e] = A_e^T B_e over each expert's rows ([E, M, N] fp32).
+// Routing-weight partials the dH kernel writes per row and N tile.
+int bwd_dh_parts_per_tile();
 cudaError_t launch_bwd_dh(const moe_config_t& c, const void* dout_perm, const int32_t* offsets, const void* wd,
                           const void* G, const void* U, const void* H, const float* row_scale, void* dG, void* dU,
                           float* dw_part, cudaStream_t s, const Ctx& ctx);

@@ -258,6 +258,19 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   return cuda_status(e);
 }
 
+moe_status_t moe_gather_rows(const void* src, int64_t n_src, const int32_t* idx, int64_t n, int64_t row_bytes,
+                             void* dst, moe_stream_t stream) {
+  if (n < 0 || n_src < 0 || row_bytes <= 0 || row_bytes % 16 != 0 || n > ((int64_t)1 << 31) ||
+      n_src > ((int64_t)1 << 31))
+    return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!src || !idx || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  moe_status_t st = get_ctx(ctx);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_gather_index(src, idx, n, n_src, row_bytes, dst, stream, ctx));
+}
+
 moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
                               moe_stream_t stream) {
   moe_status_t st = check_config(cfg);
@@ -713,7 +726,7 @@ TrainLayout train_layout_of(const moe_config_t& c) {
   L.dy_perm = take(rows * c.d * 2);
   L.dg = take(rows * c.f * 2);
   L.du = take(rows * c.f * 2);
-  L.dw_part = take(rows * (size_t)(c.f / 256) * 2 * 4);
+  L.dw_part = take(rows * (size_t)(c.f / 256) * bwd_dh_parts_per_tile() * 4);
   L.dlogits = take((size_t)c.T * c.E * 4);
   L.dweight = take((size_t)c.T * c.top_k * 4);
   L.dx32 = take((size_t)c.T * c.d * 4);
@@ -809,7 +822,7 @@ moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const vo
   const float* row_scale = reinterpret_cast<const float*>(w8 + L.row_scale);
   float* dw_part = reinterpret_cast<float*>(w8 + TL.dw_part);
   float* dx32 = reinterpret_cast<float*>(w8 + TL.dx32);
-  const int n_parts = (int)(c.f / 256) * 2;  // two column halves per dH tile
+  const int n_parts = (int)(c.f / 256) * bwd_dh_parts_per_tile();
   cudaError_t e = launch_bwd_gather(c, dout, perm, offsets, row_scale, w8 + TL.dout_perm, w8 + TL.dy_perm, stream, ctx);
   if (e == cudaSuccess)
     e = launch_bwd_dh(c, w8 + TL.dout_perm, offsets, w_down, w8 + TL.g, w8 + TL.u, w8 + L.h, row_scale, w8 + TL.dg,

@@ -1,0 +1,130 @@
+"""Expert parallelism: each rank owns E/world experts and exchanges token rows.
+
+"Expert parallelism vs. tensor parallelism" (moe_layer_ep_forward): every rank
+routes its own tokens, sends each token row to the rank owning the chosen
+expert (all-to-all), runs its own experts on what it receives, and sends the
+expert outputs back (all-to-all) for the weighted combine in token order.
+
+Here the send side needs no extra permutation: the dispatch already groups a
+rank's kept rows by expert, and the experts of one destination rank are
+contiguous, so destination q's rows are one slice of x_perm.  The receive
+side regroups rows from rank-major (as the all-to-all delivers them) to
+expert-major for the grouped GEMM, and back again for the return trip, with
+moe_gather_rows.  Routing weights stay on the source rank: experts return
+unweighted outputs and the source's combine applies the weights.
+
+The phases (ep_prepare, ep_plan, ep_experts, ep_finish) are separate so that a
+caller can run the exchanges with any transport; layer_forward_ep runs them
+with torch.distributed (NCCL on GPUs).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from . import Config, combine, dispatch, expert_ffn, gather_rows, router_topk
+
+
+def owned_experts(rank: int, world: int, E: int = 8):
+    """Experts of rank `rank`: a contiguous block of E / world."""
+    if world < 1 or E % world:
+        raise ValueError(f"world size {world} must divide E = {E}")
+    n = E // world
+    return list(range(rank * n, (rank + 1) * n))
+
+
+def ep_plan(table, rank: int, world: int):
+    """Exchange plan of rank `rank` from table[p, e] = rows rank p sends to expert e.
+
+    send_splits[q]: rows this rank sends to rank q (slices of its x_perm, in order);
+    recv_splits[p]: rows it receives from rank p.  Received rows are rank-major
+    and, within a source, expert-major; `fwd` lists for every grouped
+    (expert-major, then source-major) row the received row it comes from, `inv`
+    is its inverse, and `offsets` [E + 1] bound the grouped rows of each expert
+    (empty for experts of other ranks)."""
+    table = np.asarray(table, dtype=np.int64)
+    E = table.shape[1]
+    mine = owned_experts(rank, world, E)
+    n = len(mine)
+    send = [int(table[rank, q * n:(q + 1) * n].sum()) for q in range(world)]
+    recv = [int(table[p, mine].sum()) for p in range(world)]
+    start = np.zeros((world, n), dtype=np.int64)
+    pos = 0
+    for p in range(world):
+        for j, e in enumerate(mine):
+            start[p, j] = pos
+            pos += table[p, e]
+    fwd = np.empty(pos, dtype=np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    g = 0
+    for e in range(E):
+        offsets[e] = g
+        if e in mine:
+            j = mine.index(e)
+            for p in range(world):
+                c = int(table[p, e])
+                fwd[g:g + c] = np.arange(start[p, j], start[p, j] + c, dtype=np.int32)
+                g += c
+    offsets[E] = g
+    inv = np.empty_like(fwd)
+    inv[fwd] = np.arange(fwd.size, dtype=np.int32)
+    return {"send_splits": send, "recv_splits": recv, "fwd": fwd, "inv": inv, "offsets": offsets, "mine": mine}
+
+
+def ep_prepare(cfg: Config, x, w_router, logit_bias=None, stream=None):
+    """Route and group this rank's tokens; counts_kept [E] is what the table gathers."""
+    idx, w, _ = router_topk(cfg, x, w_router, logit_bias, stream=stream)
+    disp = dispatch(cfg, x, idx, w, stream=stream)
+    return {"idx": idx, "w": w, "disp": disp, "counts": disp["counts_kept"]}
+
+
+def ep_experts(cfg: Config, x_recv, plan, w_gate, w_up, w_down, stream=None):
+    """Run this rank's experts on the received rows; returns their (unweighted)
+    outputs in received order, fp32 [n_recv, d]."""
+    n = int(plan["offsets"][-1])
+    dev = x_recv.device
+    if n == 0:
+        return torch.empty((0, cfg.d), dtype=torch.float32, device=dev)
+    # the grouped GEMM reads up to T * top_k rows: size its buffers for the received rows
+    t_e = (n + cfg.top_k - 1) // cfg.top_k
+    cfg_e = Config(t_e, cfg.d, cfg.f, E=cfg.E, top_k=cfg.top_k, capacity_factor=float("inf"), dtype=cfg.dtype)
+    x_grp = torch.empty((t_e * cfg.top_k, cfg.d), dtype=x_recv.dtype, device=dev)
+    gather_rows(x_recv, torch.from_numpy(plan["fwd"]).to(dev), out=x_grp[:n], stream=stream)
+    offsets = torch.from_numpy(plan["offsets"]).to(dev)
+    _, y_grp = expert_ffn(cfg_e, x_grp, offsets, w_gate, w_up, w_down, None, stream=stream)
+    return gather_rows(y_grp, torch.from_numpy(plan["inv"]).to(dev), stream=stream)
+
+
+def ep_finish(cfg: Config, y_back, state, stream=None):
+    """Weighted combine of the returned expert outputs, one row per kept slot in
+    this rank's x_perm order (the combine reads only those slots)."""
+    return combine(cfg, y_back, state["disp"]["slot_of"], state["w"], weights_applied=False, stream=stream)
+
+
+def _all_to_all_rows(send, send_splits, recv_splits, group=None):
+    out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype, device=send.device)
+    dist.all_to_all_single(out, send.contiguous(), recv_splits, send_splits, group=group)
+    return out
+
+
+def gather_table(counts, group=None):
+    """table[p, e] = counts of rank p, on the host."""
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(counts) for _ in range(world)]
+    dist.all_gather(parts, counts.contiguous(), group=group)
+    return torch.stack(parts).cpu().numpy()
+
+
+def layer_forward_ep(cfg: Config, x, w_router, w_gate, w_up, w_down, logit_bias=None, group=None, stream=None):
+    """The layer with expert parallelism over the ranks of `group`: this rank's
+    tokens in, this rank's output rows out.  w_gate/w_up/w_down hold all E
+    experts' layout; only this rank's experts are read."""
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    st = ep_prepare(cfg, x, w_router, logit_bias, stream=stream)
+    plan = ep_plan(gather_table(st["counts"], group), rank, world)
+    n_send = sum(plan["send_splits"])
+    x_recv = _all_to_all_rows(st["disp"]["x_perm"][:n_send], plan["send_splits"], plan["recv_splits"], group)
+    y_recv = ep_experts(cfg, x_recv, plan, w_gate, w_up, w_down, stream=stream)
+    y_back = _all_to_all_rows(y_recv, plan["recv_splits"], plan["send_splits"], group)
+    return ep_finish(cfg, y_back, st, stream=stream)

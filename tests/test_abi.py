@@ -203,3 +203,14 @@ def test_shard_dispatch_arguments_checked_before_launch(moe):
     assert moe.STATUS[f(c.ref, 10, ok, 2, 0, None, ok, ok, ok, ok, ok, ok, ok, ok, None, ok, ws - 1, None)] == \
         "MOE_ERR_WORKSPACE"
     assert moe.STATUS[moe.lib.moe_route_counts(c.ref, ok, None, None)] == "MOE_ERR_INVALID_ARG"
+
+
+def test_gather_rows_arguments_checked_before_launch(moe):
+    P = ctypes.c_void_p
+    ok = P(256)
+    f = moe.lib.moe_gather_rows
+    assert f(ok, 10, ok, 0, 16, ok, None) == 0  # nothing to copy
+    assert moe.STATUS[f(ok, 10, ok, 4, 24, ok, None)] == "MOE_ERR_INVALID_ARG"  # row not a multiple of 16 bytes
+    assert moe.STATUS[f(ok, 10, ok, -1, 16, ok, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[f(None, 10, ok, 4, 16, ok, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[f(P(258), 10, ok, 4, 16, ok, None)] == "MOE_ERR_INVALID_ARG"  # misaligned source

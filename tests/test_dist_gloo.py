@@ -129,3 +129,74 @@ def test_three_gloo_ranks_shard_the_global_capacity():
         assert np.array_equal(res[r][1], want_table)
     kept = np.concatenate([res[r][2] for r in range(3)])
     assert np.array_equal(kept, ref["slot_of"] >= 0)
+
+
+def _ep_worker(rank, world, port, q):
+    # the exchange plan and the two all-to-alls of expert parallelism, carrying token ids
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import oracle
+    from sparse_moe_layer_07_b200.expert_parallel import _all_to_all_rows, ep_plan, gather_table
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        idx, w, cap, per = _ep_routing(oracle, world, rank)
+        disp = oracle.dispatch(idx, w, 8, cap)
+        table = gather_table(torch.from_numpy(disp["counts_kept"].astype(np.int32)))
+        plan = ep_plan(table, rank, world)
+        # each row carries (source rank, token, expert)
+        n = disp["n_kept"]
+        experts = np.repeat(np.arange(8), disp["counts_kept"])
+        rows = torch.from_numpy(np.stack([np.full(n, rank), disp["perm"], experts], 1).astype(np.int64))
+        recv = _all_to_all_rows(rows[:sum(plan["send_splits"])], plan["send_splits"], plan["recv_splits"])
+        grouped = recv.numpy()[plan["fwd"]]
+        back = _all_to_all_rows(torch.from_numpy(grouped[plan["inv"]]), plan["recv_splits"], plan["send_splits"])
+        q.put((rank, table, grouped, plan["offsets"], back.numpy(), rows.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _ep_routing(oracle, world, rank):
+    rng = np.random.default_rng(40 + rank)
+    T, d = 50, 16
+    x = rng.standard_normal((T, d))
+    wr = np.random.default_rng(39).standard_normal((8, d))
+    lg = oracle.router_logits(x, wr, np.array([1.0, 0.5, 0, 0, 0, 0, 0, -1.0]))
+    idx, w = oracle.top2_softmax(lg)
+    return idx, w, oracle.capacity(T, 2, 8, 1.25), T
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_exchange_on_gloo_ranks(world):
+    import oracle
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r = q.get(timeout=120)
+        res[r[0]] = r
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    n_own = 8 // world
+    for rank in range(world):
+        _, table, grouped, offsets, back, sent = res[rank]
+        # grouped rows of each own expert: every source's kept tokens of that expert, source-major, token order
+        for e in range(rank * n_own, (rank + 1) * n_own):
+            want = []
+            for src in range(world):
+                idx, w, cap, _ = _ep_routing(oracle, world, src)
+                d = oracle.dispatch(idx, w, 8, cap)
+                toks = d["perm"][d["offsets"][e]:d["offsets"][e + 1]]
+                want += [(src, int(t), e) for t in toks]
+            got = [tuple(int(v) for v in r) for r in grouped[offsets[e]:offsets[e + 1]]]
+            assert got == want, (rank, e)
+        assert all(offsets[e + 1] == offsets[e] for e in range(8) if e // n_own != rank)
+        # the return trip puts every row back where this rank sent it from
+        assert np.array_equal(back, sent[:back.shape[0]]) and back.shape[0] == sent.shape[0]
