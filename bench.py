@@ -198,18 +198,25 @@ def reference_arm(args, w):
     per_step = args.ref_tokens
     for i in range(args.warmup):
         oracle_sample(w, host, x, per_step, 1000 + i)
-    tot, ntok = 0.0, 0
+    # Each step is a few seconds of fp64 work on the host (the expert matrices of the
+    # sampled tokens are widened to fp64 per call); steps stop once the next one would
+    # pass the wall-clock budget, so a long --steps still ends within a few minutes.
+    tot, ntok, done = 0.0, 0, 0
     for i in range(args.steps):
+        if done and tot + tot / done > args.ref_budget_s:
+            break
         t, n = oracle_sample(w, host, x, per_step, i)
         tot += t
         ntok += n
+        done += 1
     value = ntok / tot
     cores = blas_threads()
     sample = (f"oracle (fp64 numpy) per step: router, top-2 and dispatch over all T={w.T} tokens, "
-              f"expert FFN and combine for {per_step} seeded tokens")
+              f"expert FFN and combine for {per_step} seeded tokens; {done} of {args.steps} requested steps "
+              f"timed (wall-clock budget {args.ref_budget_s:.0f} s)")
     line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+            "n_gpus": args.gpus, "steps": done, "steps_requested": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * tot / done, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
@@ -233,6 +240,7 @@ def main():
     ap.add_argument("--workload", default="grok_prefill", choices=sorted(configs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per reference-arm step")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0, help="wall-clock budget of the reference arm's steps")
     ap.add_argument("--cpu-tokens", type=int, default=64, help="tokens in the CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
@@ -314,9 +322,10 @@ def main():
     if fused:
         buf["dc_ws"] = torch.empty(moe.lib.moe_expert_down_combine_workspace_size(cfg.ref), dtype=torch.uint8,
                                    device=dev)
-    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes);
+    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes
+    # and the partial sum);
     # fused: router 1, dispatch 3 + gather 1, gate/up 1, zero + down + rounding 3 (9)
-    launches_per_step = 10 if args.int8 else (9 if fused else 8)
+    launches_per_step = 11 if args.int8 else (9 if fused else 8)
 
     def step(ev=None):
         if ev:

@@ -18,8 +18,20 @@
 namespace moe {
 namespace {
 
+// y of a slot = sum over p < n_parts of y[p * part_stride + slot * d + ...], parts
+// added in order (K-split partials of the 8-bit down pass; 1 part otherwise).
+__device__ __forceinline__ float4 slot_row(const float* y, int n_parts, int64_t part_stride, int64_t off) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(y + off));
+  for (int p = 1; p < n_parts; ++p) {
+    const float4 b = __ldg(reinterpret_cast<const float4*>(y + p * part_stride + off));
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+  }
+  return a;
+}
+
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot_of,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, int n_parts, int64_t part_stride,
+                                                     const int32_t* __restrict__ slot_of,
                                                      const float* __restrict__ topk_w, int weights_applied, int64_t T,
                                                      int64_t d, int64_t max_slot, void* __restrict__ out, int* err) {
   const int64_t nvec = d / 4;  // float4 groups per row
@@ -37,16 +49,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       c0 = wt.x;
       c1 = wt.y;
     }
-    const float4* y0 = reinterpret_cast<const float4*>(y + (int64_t)(s0 < 0 ? 0 : s0) * d);
-    const float4* y1 = reinterpret_cast<const float4*>(y + (int64_t)(s1 < 0 ? 0 : s1) * d);
+    const int64_t r0 = (int64_t)(s0 < 0 ? 0 : s0) * d, r1 = (int64_t)(s1 < 0 ? 0 : s1) * d;
     for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
       if (s0 >= 0) {
-        const float4 p = __ldg(y0 + v);
+        const float4 p = slot_row(y, n_parts, part_stride, r0 + 4 * v);
         a.x += c0 * p.x; a.y += c0 * p.y; a.z += c0 * p.z; a.w += c0 * p.w;
       }
       if (s1 >= 0) {
-        const float4 p = __ldg(y1 + v);
+        const float4 p = slot_row(y, n_parts, part_stride, r1 + 4 * v);
         a.x += c1 * p.x; a.y += c1 * p.y; a.z += c1 * p.z; a.w += c1 * p.w;
       }
       if (kBf16Out) {
@@ -111,18 +122,18 @@ cudaError_t launch_round_out(const moe_config_t& c, const float* out32, void* ou
 
 cudaError_t launch_combine(const moe_config_t& c, const float* y, const int32_t* slot_of,
                            const float* topk_w, int weights_applied, void* out, cudaStream_t s,
-                           const Ctx& ctx) {
+                           const Ctx& ctx, int n_parts, int64_t part_stride) {
   if (c.T == 0) return cudaSuccess;
   int64_t blocks = c.T;
   const int64_t cap_blocks = (int64_t)ctx.num_sms * 8;
   if (blocks > cap_blocks) blocks = cap_blocks;
   const int64_t max_slot = slot_rows(c);
   if (c.dtype == MOE_BF16)
-    combine_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(y, slot_of, topk_w, weights_applied, c.T, c.d, max_slot,
-                                                          out, ctx.err);
+    combine_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(y, n_parts, part_stride, slot_of, topk_w, weights_applied,
+                                                          c.T, c.d, max_slot, out, ctx.err);
   else
-    combine_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(y, slot_of, topk_w, weights_applied, c.T, c.d, max_slot,
-                                                           out, ctx.err);
+    combine_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(y, n_parts, part_stride, slot_of, topk_w,
+                                                           weights_applied, c.T, c.d, max_slot, out, ctx.err);
   return cudaGetLastError();
 }
 

@@ -158,8 +158,7 @@ __device__ __forceinline__ void build_schedule(Sched& sched, const BwdArgs& args
   if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
 }
 
-__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 q = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack8_bf16(const uint4 q, float (&v)[8]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -386,19 +385,35 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         const float w = valid ? __ldg(args.row_scale + row) : 0.f;
         const int64_t base = row * args.ld + t.n0;
         float dot = 0.f;
+        // G, U, H of a 32-column chunk: 4 x 16 bytes each; the next chunk's are
+        // loaded while this one is computed, so the loads overlap the math
+        uint4 qg[4], qu[4], qh[4];
+        auto load_chunk = [&](int c, uint4 (&a)[4], uint4 (&b)[4], uint4 (&hh)[4]) {
+          const int64_t o = base + c * 32;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            a[p] = *reinterpret_cast<const uint4*>(args.G + o + p * 8);
+            b[p] = *reinterpret_cast<const uint4*>(args.U + o + p * 8);
+            hh[p] = *reinterpret_cast<const uint4*>(args.H + o + p * 8);
+          }
+        };
+        if (valid) load_chunk(c_begin, qg, qu, qh);
 #pragma unroll 1
         for (int c = c_begin; c < c_end; ++c) {
           uint32_t v[32];
           tmem_ld32(tacc + c * 32, v);
+          const bool more = c + 1 < c_end;
+          uint4 ng[4], nu[4], nh[4];
+          if (valid && more) load_chunk(c + 1, ng, nu, nh);
           tmem_wait_ld();
           if (valid) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
               const int64_t o = base + c * 32 + p * 8;
               float g[8], u[8], h[8];
-              load8_bf16(args.G + o, g);
-              load8_bf16(args.U + o, u);
-              load8_bf16(args.H + o, h);
+              unpack8_bf16(qg[p], g);
+              unpack8_bf16(qu[p], u);
+              unpack8_bf16(qh[p], h);
               uint32_t og[4], ou[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -419,6 +434,14 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
               }
               *reinterpret_cast<uint4*>(args.dG + o) = make_uint4(og[0], og[1], og[2], og[3]);
               *reinterpret_cast<uint4*>(args.dU + o) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+            }
+          }
+          if (more) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              qg[p] = ng[p];
+              qu[p] = nu[p];
+              qh[p] = nh[p];
             }
           }
         }

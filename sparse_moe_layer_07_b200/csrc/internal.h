@@ -45,7 +45,8 @@ cudaError_t launch_gather(const moe_config_t& c, const void* x, const int32_t* p
 
 cudaError_t launch_combine(const moe_config_t& c, const float* y, const int32_t* slot_of,
                            const float* topk_w, int weights_applied, void* out, cudaStream_t s,
-                           const Ctx& ctx);
+                           const Ctx& ctx,
+                           int n_parts = 1, int64_t part_stride = 0);
 
 // fp32 expert FFN on the CUDA cores (exact fp32 FMA; no TF32).
 cudaError_t launch_ffn_simt_gate_up(const moe_config_t& c, const float* x_perm,
@@ -125,7 +126,8 @@ cudaError_t launch_decode_down(const moe_config_t& c, const void* h, const int32
 // 15-bit row codes (hi/lo int8 planes + per-row scale) of the first offsets[E]
 // rows of src ([rows, K], bf16 or fp32).
 cudaError_t launch_quantize_rows(const void* src, bool src_f32, const int32_t* offsets, int64_t max_rows,
-                                 int64_t K, int8_t* hi, int8_t* lo, float* scale, int num_sms, cudaStream_t s);
+                                 int64_t K, int8_t* hi, int8_t* lo, float* scale, int num_sms, cudaStream_t s,
+                                 const int32_t* perm = nullptr, int64_t n_src = 0, int* err = nullptr);
 
 // Expert GEMMs on the int8 tensor cores: int8 weights x row-code planes.
 cudaError_t launch_i8_gate_up(const moe_config_t& c, const int8_t* x_hi, const int8_t* x_lo,

@@ -594,9 +594,12 @@ W8Layout w8_layout_of(const moe_config_t& c) {
   return L;
 }
 
-cudaError_t run_ffn_w8(const moe_config_t& c, const void* x_perm, const int32_t* offsets, const int8_t* qg,
+// x_rows: x_perm, or (with perm) x itself read by slot; y == nullptr leaves the
+// down pass's K-split partials unsummed (the layer's combine adds them in order).
+cudaError_t run_ffn_w8(const moe_config_t& c, const void* x_rows, const int32_t* offsets, const int8_t* qg,
                        const float* sg, const int8_t* qu, const float* su, const int8_t* qd, const float* sd,
-                       const float* row_scale, float* y, uint8_t* ws, cudaStream_t s, const Ctx& ctx) {
+                       const float* row_scale, float* y, uint8_t* ws, cudaStream_t s, const Ctx& ctx,
+                       const int32_t* perm = nullptr) {
   const W8Layout L = w8_layout_of(c);
   const int64_t rows = slot_rows(c);
   int8_t* x_hi = reinterpret_cast<int8_t*>(ws + L.x_hi);
@@ -606,13 +609,19 @@ cudaError_t run_ffn_w8(const moe_config_t& c, const void* x_perm, const int32_t*
   int8_t* h_hi = reinterpret_cast<int8_t*>(ws + L.h_hi);
   int8_t* h_lo = reinterpret_cast<int8_t*>(ws + L.h_lo);
   float* h_sc = reinterpret_cast<float*>(ws + L.h_scale);
-  cudaError_t e = launch_quantize_rows(x_perm, false, offsets, rows, c.d, x_hi, x_lo, x_sc, ctx.num_sms, s);
+  cudaError_t e = launch_quantize_rows(x_rows, false, offsets, rows, c.d, x_hi, x_lo, x_sc, ctx.num_sms, s, perm, c.T,
+                                       ctx.err);
   if (e == cudaSuccess) e = launch_i8_gate_up(c, x_hi, x_lo, x_sc, offsets, qg, sg, qu, su, h, s, ctx);
   if (e == cudaSuccess) e = launch_quantize_rows(h, true, offsets, rows, c.f, h_hi, h_lo, h_sc, ctx.num_sms, s);
   float* y_parts = reinterpret_cast<float*>(ws + L.y_parts);
   if (e == cudaSuccess) e = launch_i8_down(c, h_hi, h_lo, h_sc, offsets, qd, sd, row_scale, y_parts, s, ctx);
-  if (e == cudaSuccess) e = launch_sum_partials(c, y_parts, offsets, y, s, ctx);
+  if (e == cudaSuccess && y) e = launch_sum_partials(c, y_parts, offsets, y, s, ctx);
   return e;
+}
+
+// The K-split partials of the 8-bit down pass, for a combine that sums them.
+const float* w8_partials(const moe_config_t& c, const uint8_t* ws) {
+  return reinterpret_cast<const float*>(ws + w8_layout_of(c).y_parts);
 }
 
 }  // namespace
@@ -667,17 +676,18 @@ moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const 
   int32_t* perm = reinterpret_cast<int32_t*>(w8 + L.perm);
   int32_t* slot_of = reinterpret_cast<int32_t*>(w8 + L.slot_of);
   float* row_scale = reinterpret_cast<float*>(w8 + L.row_scale);
-  void* x_perm = w8 + L.x_perm;
-  float* y = reinterpret_cast<float*>(w8 + L.y);
   cudaError_t e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, stream, ctx);
   if (e == cudaSuccess)
     e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, route, route + c.E, offsets, perm, slot_of, row_scale,
                         reinterpret_cast<int32_t*>(w8 + L.disp), stats, stream, ctx);
-  if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, x_perm, stream, ctx);
+  // x rows are coded straight from x by slot (no x_perm), and the combine adds the
+  // down pass's K-split partials itself, in the order the partial sum would
   if (e == cudaSuccess)
-    e = run_ffn_w8(c, x_perm, offsets, q_gate, s_gate, q_up, s_up, q_down, s_down, row_scale, y, w8 + L.total, stream,
-                   ctx);
-  if (e == cudaSuccess) e = launch_combine(c, y, slot_of, topk_w, 1, out, stream, ctx);
+    e = run_ffn_w8(c, x, offsets, q_gate, s_gate, q_up, s_up, q_down, s_down, row_scale, nullptr, w8 + L.total,
+                   stream, ctx, perm);
+  if (e == cudaSuccess)
+    e = launch_combine(c, w8_partials(c, w8 + L.total), slot_of, topk_w, 1, out, stream, ctx, down_splits(c),
+                       slot_rows(c) * c.d);
   return cuda_status(e);
 }
 

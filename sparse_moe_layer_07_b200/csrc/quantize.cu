@@ -82,16 +82,27 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
 }
 
+// Row r of the source is src row perm[r] when perm is given (rows gathered on
+// the fly, e.g. x by slot), else src row r.
 template <typename Tin>
-__global__ void __launch_bounds__(1024) quantize_rows_kernel(const Tin* __restrict__ src, const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(1024) quantize_rows_kernel(const Tin* __restrict__ src, const int32_t* __restrict__ perm,
+                                                           int64_t n_src, const int32_t* __restrict__ offsets,
                                                            int64_t max_rows, int64_t K, int8_t* __restrict__ hi,
-                                                           int8_t* __restrict__ lo, float* __restrict__ scale) {
+                                                           int8_t* __restrict__ lo, float* __restrict__ scale, int* err) {
   __shared__ float s_max[32];
   int64_t n = offsets[8];
   if (n < 0 || n > max_rows) n = 0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
-    const Tin* row = src + r * K;
+    int64_t sr = r;
+    if (perm) {
+      sr = perm[r];
+      if (sr < 0 || sr >= n_src) {
+        if (threadIdx.x == 0) flag_error(err, MOE_DEVERR_SLOT_INDEX);
+        continue;  // uniform over the block: every thread skips this row
+      }
+    }
+    const Tin* row = src + sr * K;
     float m = 0.f;
     for (int64_t k = 4 * (int64_t)threadIdx.x; k < K; k += 4 * (int64_t)blockDim.x) {
       float v[4];
@@ -128,16 +139,17 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const Tin* __restri
 }  // namespace
 
 cudaError_t launch_quantize_rows(const void* src, bool src_f32, const int32_t* offsets, int64_t max_rows,
-                                 int64_t K, int8_t* hi, int8_t* lo, float* scale, int num_sms, cudaStream_t s) {
+                                 int64_t K, int8_t* hi, int8_t* lo, float* scale, int num_sms, cudaStream_t s,
+                                 const int32_t* perm, int64_t n_src, int* err) {
   if (max_rows == 0) return cudaSuccess;
   int64_t blocks = max_rows < (int64_t)num_sms * 4 ? max_rows : (int64_t)num_sms * 4;
   const int threads = K >= 16384 ? 1024 : 256;  // long rows (H) get more threads per row
   if (src_f32)
-    quantize_rows_kernel<float><<<(unsigned)blocks, threads, 0, s>>>(static_cast<const float*>(src), offsets,
-                                                                     max_rows, K, hi, lo, scale);
+    quantize_rows_kernel<float><<<(unsigned)blocks, threads, 0, s>>>(static_cast<const float*>(src), perm, n_src,
+                                                                     offsets, max_rows, K, hi, lo, scale, err);
   else
     quantize_rows_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(src), offsets, max_rows, K, hi, lo, scale);
+        static_cast<const __nv_bfloat16*>(src), perm, n_src, offsets, max_rows, K, hi, lo, scale, err);
   return cudaGetLastError();
 }
 
