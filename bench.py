@@ -224,6 +224,25 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+def hbm_steps(w, n_kept, per_kernel, fused, peaks):
+    """Achieved bandwidth of the memory-bound steps from their algorithmic bytes:
+    router T*d*b + E*d*b + 16*T; dispatch (3 kernels) + gather 8*T + 12*N + 2*N*d*b;
+    combine 4*N*d + 8*T + T*d*b (in the fused path the combine is inside the down pass)."""
+    b = 2 if w.storage == "bf16" else 4
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    out = {}
+    items = {"router": w.T * w.d * b + w.E * w.d * b + 16 * w.T,
+             "dispatch": 8 * w.T + 12 * n_kept + 2 * n_kept * w.d * b}
+    if not fused:
+        items["combine"] = 4 * n_kept * w.d + 8 * w.T + w.T * w.d * b
+    for name, nbytes in items.items():
+        ms = per_kernel.get(name, 0.0)
+        if ms > 0:
+            gbs = nbytes / (ms / 1000.0) / 1e9
+            out[name] = {"bytes": nbytes, "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm}
+    return out
+
+
 def workload_config(w):
     return {"workload": w.name, "T": w.T, "d": w.d, "f": w.f, "E": w.E, "top_k": w.top_k,
             "capacity_factor": w.capacity_factor, "logit_bias": list(w.logit_bias) if w.logit_bias else None,
@@ -424,6 +443,7 @@ def main():
             "config": dict(workload_config(w), expert_weights="int8" if args.int8 else w.storage), "tflops": tflops,
             "tensor_frac_layer": tflops / peak,
             "kernels_ms": per_kernel,
+            "hbm_steps": hbm_steps(w, n_kept, per_kernel, fused, peaks),
             "path": ("down-combine fused: down sums into token order (its time includes the zeroing and "
                      "rounding passes; combine 0)") if fused else "separate down and combine",
             "counts_kept": counts_kept, "n_kept": n_kept,

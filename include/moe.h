@@ -1,6 +1,8 @@
 /*
- * moe.h -- C ABI of a B200 (sm_100a) implementation of the forward pass of a
- * Grok-1-style sparse mixture-of-experts SwiGLU FFN layer.
+ * moe.h -- C ABI of a B200 (sm_100a) implementation of a Grok-1-style sparse
+ * mixture-of-experts SwiGLU FFN layer: the forward pass (bf16 and fp32, with a
+ * weight-streaming path for small batches and an int8-weight path), its
+ * backward pass for training, and the row exchange helpers of multi-rank use.
  *
  * The operation follows the page "How does Grok-1 use a mixture-of-experts
  * design?" (n4n.ai):
@@ -23,8 +25,9 @@
  *
  * Conventions for every entry point:
  *   - Pointers named *_host are host memory; every other buffer pointer is
- *     device memory owned by the caller.  The library never allocates, frees
- *     or keeps a pointer after a call returns.
+ *     device memory owned by the caller.  The library never allocates or frees
+ *     device memory (moe_dispatch_noalloc uses one fixed array inside the
+ *     library) and keeps no pointer after a call returns.
  *   - Tensors are dense row-major.  Buffers must be 16-byte aligned.
  *   - Work is enqueued on `stream` (a cudaStream_t); calls return before the
  *     GPU finishes, except moe_layer_forward_host, moe_layer_forward_host_batches
@@ -160,6 +163,14 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const 
  * and counts_kept[e] = min(counts_raw[e], max(capacity - prior[e], 0)).
  * capacity is the global one (moe_capacity of the whole batch's config);
  * cfg->T is this shard's token count.  Deterministic, no atomics. */
+MOE_API moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
+                              moe_stream_t stream);
+MOE_API moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const int32_t* shard_counts,
+                                int32_t n_shards, int32_t shard, const void* x, const int32_t* topk_idx,
+                                const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
+                                int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
+                                void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Row gather, dst[i, :] = src[idx[i], :] for i < n: rows of row_bytes bytes
  * (a multiple of 16), src holding n_src rows (device memory; idx device int32).
  * Used to regroup rows between the expert-major order of a rank's own experts
@@ -168,14 +179,6 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const 
  * index outside [0, n_src) skips its row and sets MOE_DEVERR_SLOT_INDEX. */
 MOE_API moe_status_t moe_gather_rows(const void* src, int64_t n_src, const int32_t* idx, int64_t n,
                              int64_t row_bytes, void* dst, moe_stream_t stream);
-
-MOE_API moe_status_t moe_route_counts(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts,
-                              moe_stream_t stream);
-MOE_API moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const int32_t* shard_counts,
-                                int32_t n_shards, int32_t shard, const void* x, const int32_t* topk_idx,
-                                const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
-                                int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
-                                void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* SwiGLU expert FFN over the grouped rows ("Expert implementation: SwiGLU at
  * scale", SwiGLUExpert / FusedSwiGLUExpert), for each expert e and each row r
