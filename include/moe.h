@@ -369,6 +369,13 @@ MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void* x
                                           int32_t* offsets, int32_t* perm, int32_t* slot_of,
                                           float* row_scale, void* x_perm, moe_stream_t stream);
 
+/* Check of the bounded waits every pipelined kernel uses: one block waits on an
+ * mbarrier that nothing completes, giving up after limit_ns nanoseconds
+ * (1 us .. 1 s) and setting MOE_DEVERR_TIMEOUT in the device error word, as a
+ * kernel whose pipeline stalled would.  The context stays usable; read the bit
+ * with moe_get_device_error. */
+MOE_API moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t stream);
+
 /* Waits for the current device, returns the device error word (MOE_DEVERR_*
  * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.
  * Returns MOE_ERR_DEVICE_CHECK when the word is non-zero, else MOE_OK. */

@@ -78,6 +78,7 @@ def _load():
         "moe_workspace_size_train": ([cfgp], sz),
         "moe_route_counts": ([cfgp, P, P, P], ctypes.c_int),
         "moe_gather_rows": ([P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int64, P, P], ctypes.c_int),
+        "moe_check_bounded_wait": ([ctypes.c_int64, P], ctypes.c_int),
         "moe_dispatch_shard": ([cfgp, ctypes.c_int64, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, P, P, P,
                                 P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_train": ([cfgp, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),

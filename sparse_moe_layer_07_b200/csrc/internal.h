@@ -99,6 +99,10 @@ constexpr int kRouterBwdChunks = 32;  // token chunks of the dW_r partial sums
 cudaError_t launch_zero_rows(const moe_config_t& c, float* out32, cudaStream_t s, const Ctx& ctx);
 cudaError_t launch_round_out(const moe_config_t& c, const float* out32, void* out, cudaStream_t s, const Ctx& ctx);
 
+// One block waits on an mbarrier nothing completes, bounded by limit_ns; sets
+// MOE_DEVERR_TIMEOUT when the wait gives up (check of the bounded-wait path).
+cudaError_t launch_wait_check(int64_t limit_ns, cudaStream_t s, const Ctx& ctx);
+
 // Argument check shared by the entry points (MOE_OK when the config is usable).
 moe_status_t validate_config(const moe_config_t* cfg);
 // Device facts of the current device (cached per device).

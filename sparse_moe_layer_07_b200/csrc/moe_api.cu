@@ -9,6 +9,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 #include "moe.h"
 
@@ -186,6 +188,15 @@ bool encode_tmap_dtype(CUtensorMap* map, const void* base, int rank, const uint6
 
 using namespace moe;
 
+namespace {
+// NVTX range around an entry point (visible in Nsight timelines; no cost
+// without a tool attached).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
+}  // namespace
+
 extern "C" {
 
 int32_t moe_abi_version(void) { return 1; }
@@ -225,6 +236,7 @@ size_t moe_workspace_size(const moe_config_t* cfg) {
 
 moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
                              float* logits, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  Range range_("moe_router_topk");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -240,6 +252,7 @@ moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void*
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const float* topk_w,
                           int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets, int32_t* perm, int32_t* slot_of,
                           float* row_scale, void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_dispatch");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!topk_idx || !topk_w || !counts_raw || !counts_kept || !offsets || !perm || !slot_of || !row_scale)
@@ -260,6 +273,7 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
 
 moe_status_t moe_gather_rows(const void* src, int64_t n_src, const int32_t* idx, int64_t n, int64_t row_bytes,
                              void* dst, moe_stream_t stream) {
+  Range range_("moe_gather_rows");
   if (n < 0 || n_src < 0 || row_bytes <= 0 || row_bytes % 16 != 0 || n > ((int64_t)1 << 31) ||
       n_src > ((int64_t)1 << 31))
     return MOE_ERR_INVALID_ARG;
@@ -286,6 +300,7 @@ moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const
                                 const float* topk_w, int32_t* counts_raw, int32_t* counts_kept, int32_t* offsets,
                                 int32_t* perm, int32_t* slot_of, float* row_scale, void* x_perm, void* ws,
                                 size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_dispatch_shard");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (capacity < 0 || n_shards < 1 || shard < 0 || shard >= n_shards || !shard_counts) return MOE_ERR_INVALID_ARG;
@@ -307,6 +322,7 @@ moe_status_t moe_dispatch_shard(const moe_config_t* cfg, int64_t capacity, const
 
 moe_status_t moe_expert_gate_up(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
                                 const void* w_gate, const void* w_up, void* h, moe_stream_t stream) {
+  Range range_("moe_expert_gate_up");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -319,6 +335,7 @@ moe_status_t moe_expert_gate_up(const moe_config_t* cfg, const void* x_perm, con
 
 moe_status_t moe_expert_down(const moe_config_t* cfg, const void* h, const int32_t* offsets, const void* w_down,
                              const float* row_scale, float* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_expert_down");
   (void)ws;
   (void)ws_bytes;
   moe_status_t st = check_config(cfg);
@@ -339,6 +356,7 @@ size_t moe_expert_down_combine_workspace_size(const moe_config_t* cfg) {
 moe_status_t moe_expert_down_combine(const moe_config_t* cfg, const void* h, const int32_t* offsets,
                                      const void* w_down, const float* row_scale, const int32_t* perm, void* out,
                                      void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_expert_down_combine");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -367,6 +385,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const i
 
 moe_status_t moe_combine(const moe_config_t* cfg, const float* y, const int32_t* slot_of, const float* topk_w,
                          int32_t weights_applied, void* out, moe_stream_t stream) {
+  Range range_("moe_combine");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -436,6 +455,7 @@ static moe_status_t check_layer_args(const moe_config_t* cfg, const void* w_rout
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
                                const void* w_gate, const void* w_up, const void* w_down, void* out, int32_t* stats,
                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_forward");
   moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -449,6 +469,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
 moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host, const void* w_router,
                                     const float* logit_bias, const void* w_gate, const void* w_up, const void* w_down,
                                     void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_forward_host");
   moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -485,6 +506,7 @@ moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_b
                                             const void* w_router, const float* logit_bias, const void* w_gate,
                                             const void* w_up, const void* w_down, void* const* out_host, void* ws,
                                             size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_forward_host_batches");
   moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (n_batches < 0) return MOE_ERR_INVALID_ARG;
@@ -542,6 +564,7 @@ moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_b
 
 moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
                                moe_stream_t stream) {
+  Range range_("moe_quantize_int8");
   moe_status_t st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
@@ -643,6 +666,7 @@ moe_status_t moe_expert_ffn_w8(const moe_config_t* cfg, const void* x_perm, cons
                                const int8_t* q_gate, const float* s_gate, const int8_t* q_up, const float* s_up,
                                const int8_t* q_down, const float* s_down, const float* row_scale, float* y, void* ws,
                                size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_expert_ffn_w8");
   moe_status_t st = check_w8(cfg, q_gate, s_gate, q_up, s_up, q_down, s_down);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
@@ -658,6 +682,7 @@ moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const 
                                   const float* logit_bias, const int8_t* q_gate, const float* s_gate,
                                   const int8_t* q_up, const float* s_up, const int8_t* q_down, const float* s_down,
                                   void* out, int32_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_forward_w8");
   moe_status_t st = check_w8(cfg, q_gate, s_gate, q_up, s_up, q_down, s_down);
   if (st != MOE_OK) return st;
   if (!w_router || !aligned16(w_router) || (logit_bias && !aligned16(logit_bias))) return MOE_ERR_INVALID_ARG;
@@ -689,6 +714,14 @@ moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const 
     e = launch_combine(c, w8_partials(c, w8 + L.total), slot_of, topk_w, 1, out, stream, ctx, down_splits(c),
                        slot_rows(c) * c.d);
   return cuda_status(e);
+}
+
+moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  moe_status_t st = get_ctx(ctx);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_wait_check(limit_ns, stream, ctx));
 }
 
 moe_status_t moe_get_device_error(int32_t* code, int32_t clear) {
@@ -762,6 +795,7 @@ size_t moe_workspace_size_train(const moe_config_t* cfg) {
 moe_status_t moe_layer_forward_train(const moe_config_t* cfg, const void* x, const void* w_router,
                                      const float* logit_bias, const void* w_gate, const void* w_up,
                                      const void* w_down, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_forward_train");
   moe_status_t st = check_layer_args(cfg, w_router, logit_bias, w_gate, w_up, w_down, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (!train_supported(*cfg)) return MOE_ERR_UNSUPPORTED;
@@ -799,6 +833,7 @@ moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const vo
                                 const void* w_up, const void* w_down, const void* dout, void* dx, float* dw_router,
                                 float* dbias, float* dw_gate, float* dw_up, float* dw_down, void* ws,
                                 size_t ws_bytes, moe_stream_t stream) {
+  Range range_("moe_layer_backward");
   moe_status_t st = check_layer_args(cfg, w_router, nullptr, w_gate, w_up, w_down, ws, ws_bytes);
   if (st != MOE_OK) return st;
   if (!train_supported(*cfg)) return MOE_ERR_UNSUPPORTED;

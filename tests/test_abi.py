@@ -214,3 +214,8 @@ def test_gather_rows_arguments_checked_before_launch(moe):
     assert moe.STATUS[f(ok, 10, ok, -1, 16, ok, None)] == "MOE_ERR_INVALID_ARG"
     assert moe.STATUS[f(None, 10, ok, 4, 16, ok, None)] == "MOE_ERR_INVALID_ARG"
     assert moe.STATUS[f(P(258), 10, ok, 4, 16, ok, None)] == "MOE_ERR_INVALID_ARG"  # misaligned source
+
+
+def test_bounded_wait_check_limits(moe):
+    assert moe.STATUS[moe.lib.moe_check_bounded_wait(10, None)] == "MOE_ERR_INVALID_ARG"
+    assert moe.STATUS[moe.lib.moe_check_bounded_wait(2_000_000_000, None)] == "MOE_ERR_INVALID_ARG"

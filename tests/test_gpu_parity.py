@@ -207,6 +207,21 @@ def test_all_tokens_to_two_experts_drop_and_zero():
     check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"], np.arange(256))
 
 
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    # an mbarrier nothing completes: the wait gives up after 50 ms and reports it
+    moe.get_device_error(clear=True)
+    st = moe.lib.moe_check_bounded_wait(50_000_000, None)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert moe.get_device_error(clear=True) & moe.DEVERR["TIMEOUT"]
+    w = configs.scaled(W["mid_bf16"], name="after_timeout", T=300, d=256, f=384)
+    L = LayerInputs(w)
+    g = run_steps(L)
+    ref = oracle.layer_forward(L.x, L.wr, L.wg, L.wu, L.wd, w.capacity_factor)
+    check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"], np.arange(w.T))
+    assert moe.get_device_error() == 0
+
+
 def test_bad_expert_index_sets_device_error_without_trap():
     c = moe.Config(64, 256, 384, dtype="bf16")
     idx = torch.zeros((64, 2), dtype=torch.int32, device="cuda")
