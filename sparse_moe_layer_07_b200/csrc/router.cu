@@ -49,7 +49,7 @@ __device__ __forceinline__ void finish_token(const float (&l)[kE], int64_t t, fl
 }
 
 // kTokPerWarp tokens share each W_r chunk a warp loads: 4 for large batches
-// (less L1 traffic), 1 for small ones (more warps in flight).
+// (less L1 traffic), 2 or 1 for smaller ones (more warps in flight).
 template <typename Tin, int kTokPerWarp>
 __global__ void __launch_bounds__(kWarps * 32) router_top2_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
                                                                  const float* __restrict__ bias, float* __restrict__ logits,
@@ -189,7 +189,10 @@ cudaError_t launch_router(const moe_config_t& c, const void* x, const void* wr, 
           static_cast<const float*>(x), static_cast<const float*>(wr), bias, logits, idx, w, c.d);
     return cudaGetLastError();
   }
+  // tokens per warp: as many as keep at least two blocks per SM (x is streamed
+  // once, so warps in flight set the speed; more tokens per warp share W_r loads)
   if (c.T <= (int64_t)ctx.num_sms * kWarps) return launch_router_t<1>(c, x, wr, bias, logits, idx, w, s);
+  if (c.T <= (int64_t)ctx.num_sms * kWarps * 4 * 2) return launch_router_t<2>(c, x, wr, bias, logits, idx, w, s);
   return launch_router_t<4>(c, x, wr, bias, logits, idx, w, s);
 }
 
