@@ -324,8 +324,9 @@ MOE_API moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, i
  * are the MMA's M operand and tokens its N operand, 32 per tile).
  * ws: moe_expert_ffn_w8_workspace_size bytes, laid out (256-byte aligned) as
  * x codes hi [T*2, d] int8 | lo [T*2, d] int8 | scale [T*2] fp32 | H [T*2, f]
- * fp32 | H codes hi [T*2, f] | lo [T*2, f] | scale [T*2] | up to four K-split
- * partial outputs [4, T*2, d] fp32 (summed in a fixed order into y);
+ * fp32 | H codes hi [T*2, f] | lo [T*2, f] | scale [T*2] | K-split partial
+ * outputs [s, T*2, d] fp32 (s up to 8 when T*2 <= 64*E, else 1; summed in
+ * split order into y);
  * y [T*2, d] fp32.  d must be a multiple of 256 (the down pass covers 256
  * output channels per tile). */
 MOE_API size_t moe_expert_ffn_w8_workspace_size(const moe_config_t* cfg);

@@ -461,6 +461,11 @@ def _round256(n):
     return (n + 255) // 256 * 256
 
 
+def _W8_PARTS(cfg: Config) -> int:
+    """Partial buffers the 8-bit down pass may use (up to 8 K splits at decode sizes)."""
+    return 1 if cfg.T * cfg.top_k > 64 * cfg.E else 8
+
+
 def w8_workspace_views(cfg: Config, ws):
     """Named views into the scratch of expert_ffn_w8 (layout stated in include/moe.h)."""
     rows, d, f = cfg.T * cfg.top_k, cfg.d, cfg.f
@@ -468,7 +473,7 @@ def w8_workspace_views(cfg: Config, ws):
             ("x_scale", rows * 4, torch.float32, (rows,)), ("h", rows * f * 4, torch.float32, (rows, f)),
             ("h_hi", rows * f, torch.int8, (rows, f)), ("h_lo", rows * f, torch.int8, (rows, f)),
             ("h_scale", rows * 4, torch.float32, (rows,)),
-            ("y_parts", 4 * rows * d * 4, torch.float32, (4, rows, d))]
+            ("y_parts", _W8_PARTS(cfg) * rows * d * 4, torch.float32, (_W8_PARTS(cfg), rows, d))]
     views, o = {}, 0
     for name, nbytes, dt, shape in spec:
         views[name] = ws[o:o + nbytes].view(dt).view(shape)

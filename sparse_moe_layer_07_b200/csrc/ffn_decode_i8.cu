@@ -45,10 +45,28 @@ enum Mode { kGateUp = 0, kDown = 1 };
 
 }  // namespace
 
-// K splits of the int8 down pass (see launch_i8_down).
-int down_splits(const moe_config_t& c) {
+// K splits of the int8 down pass.  With decode-sized batches (one token block
+// per expert) the down pass has only E * d / 256 tiles, too few to fill the
+// GPU evenly, so K is split into s ranges (each writing its own fp32 partial,
+// summed later in split order); s is the count in 1..kMaxDownSplits whose tile
+// count E * (d / 256) * s fills the last wave best.  Larger batches have enough
+// tiles and use one split.
+int down_splits(const moe_config_t& c, int num_sms) {
   const int64_t kb = c.f / 128;
-  return kb % 4 == 0 ? 4 : (kb % 2 == 0 ? 2 : 1);
+  if (slot_rows(c) > 64 * (int64_t)c.E) return 1;
+  const int64_t base = (int64_t)c.E * (c.d / 256);
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= kMaxDownSplits && sp <= kb; ++sp) {
+    const int64_t tiles = base * sp;
+    const int64_t waves = (tiles + num_sms - 1) / num_sms;
+    const double eff = (double)tiles / (double)(waves * num_sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = sp;
+    }
+  }
+  return best;
 }
 
 namespace {
@@ -76,8 +94,8 @@ struct I8Args {
   int64_t rows_alloc;
   int n_cb;                 // output channels / channels per tile
   int n_out;                // output channels
-  int num_kb;               // K / 128 per split
-  int ksplit;               // K splits (down: 2, each writes its own partial output)
+  int num_kb;               // K / 128 (all splits together)
+  int ksplit;               // K splits (down: each split's range writes its own partial output)
   int64_t split_stride;     // elements between the partial outputs
   void* out;                // H fp32 [rows, f] or Y fp32 [rows, d]
   int64_t ld_out;
@@ -205,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         const Tile8 t = tile8(sched, L, args.n_cb, args.ksplit, C::kChW);
-        for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+        const int kb_lo = t.ks * args.num_kb / args.ksplit, kb_hi = (t.ks + 1) * args.num_kb / args.ksplit;
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
@@ -214,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = stages + s * C::STAGE;
           mbar_arrive_expect_tx(&full[s], C::kMats * W_TILE + 2 * t.ntok * BK);
-          const int k0 = (t.ks * args.num_kb + kb) * BK;
+          const int k0 = kb * BK;
           tma_load_3d(st, &tmW0, &full[s], t.n0, k0, t.e);
           if (MODE == kGateUp)
             tma_load_3d(st + W_TILE, &tmW1, &full[s], t.n0, k0, t.e);
@@ -251,7 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d0 = tmem_base + buf * C::kAccStride;
-        for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+        const int kb_lo = t.ks * args.num_kb / args.ksplit, kb_hi = (t.ks + 1) * args.num_kb / args.ksplit;
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&full[s], ph, abort_flag)) {
@@ -266,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 32; ++kk) {
             const uint64_t b_hi = sw128_desc(p_hi + kk * 32, 16, 1024);
             const uint64_t b_lo = sw128_desc(p_lo + kk * 32, 16, 1024);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb != kb_lo || kk != 0) ? 1u : 0u;
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
               const uint64_t ad = sw128_desc(st + m * W_TILE + kk * 4096, 8192, 1024);
@@ -409,7 +429,7 @@ cudaError_t launch_sum_partials(const moe_config_t& c, const float* y_parts, con
                                 cudaStream_t s, const Ctx& ctx) {
   const int64_t rows = slot_rows(c);
   if (rows == 0) return cudaSuccess;
-  const int nsplit = down_splits(c);
+  const int nsplit = down_splits(c, ctx.num_sms);
   sum_partials_kernel<<<ctx.num_sms * 4, 256, 0, s>>>(reinterpret_cast<const float4*>(y_parts), offsets, rows,
                                                       c.d / 4, rows * c.d / 4, nsplit, reinterpret_cast<float4*>(y));
   return cudaGetLastError();
@@ -459,8 +479,8 @@ cudaError_t launch_i8_down(const moe_config_t& c, const int8_t* h_hi, const int8
   a.rows_alloc = rows;
   a.n_cb = (int)(c.d / (2 * CH));
   a.n_out = (int)c.d;
-  a.ksplit = down_splits(c);
-  a.num_kb = (int)(c.f / BK) / a.ksplit;
+  a.ksplit = down_splits(c, ctx.num_sms);
+  a.num_kb = (int)(c.f / BK);
   a.split_stride = rows * c.d;
   a.out = y_parts;
   a.ld_out = c.d;

@@ -138,8 +138,10 @@ cudaError_t launch_i8_gate_up(const moe_config_t& c, const int8_t* x_hi, const i
                               const float* x_scale, const int32_t* offsets, const int8_t* qg,
                               const float* sg, const int8_t* qu, const float* su, float* h, cudaStream_t s,
                               const Ctx& ctx);
-// K splits of the int8 down pass (1, 2 or 4).
-int down_splits(const moe_config_t& c);
+// K splits of the int8 down pass (1 .. kMaxDownSplits; each split writes an fp32
+// partial [T*k, d], summed in split order).
+constexpr int kMaxDownSplits = 8;
+int down_splits(const moe_config_t& c, int num_sms);
 // Writes down_splits(c) K-split partials [splits, T*k, d] fp32; launch_sum_partials adds them into y.
 cudaError_t launch_i8_down(const moe_config_t& c, const int8_t* h_hi, const int8_t* h_lo, const float* h_scale,
                            const int32_t* offsets, const int8_t* qd, const float* sd, const float* row_scale,

@@ -612,7 +612,7 @@ W8Layout w8_layout_of(const moe_config_t& c) {
   L.h_hi = take(rows * c.f);
   L.h_lo = take(rows * c.f);
   L.h_scale = take(rows * 4);
-  L.y_parts = take(4 * rows * c.d * 4);
+  L.y_parts = take((rows > 64 * (size_t)c.E ? 1 : kMaxDownSplits) * rows * c.d * 4);
   L.total = o;
   return L;
 }
@@ -711,8 +711,8 @@ moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const 
     e = run_ffn_w8(c, x, offsets, q_gate, s_gate, q_up, s_up, q_down, s_down, row_scale, nullptr, w8 + L.total,
                    stream, ctx, perm);
   if (e == cudaSuccess)
-    e = launch_combine(c, w8_partials(c, w8 + L.total), slot_of, topk_w, 1, out, stream, ctx, down_splits(c),
-                       slot_rows(c) * c.d);
+    e = launch_combine(c, w8_partials(c, w8 + L.total), slot_of, topk_w, 1, out, stream, ctx,
+                       down_splits(c, ctx.num_sms), slot_rows(c) * c.d);
   return cuda_status(e);
 }
 
