@@ -62,6 +62,8 @@ struct Cfg {
   static constexpr int kBarBytes = 256;
   static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + kBarBytes;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, MMA_N, false, true);
+  // an expert's last row block with at most 64 rows runs M = 64 MMAs (half the work)
+  static constexpr uint32_t IDESC_M64 = idesc_bf16_f32(64, MMA_N, false, true);
 };
 
 struct TcArgs {
@@ -248,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
         const uint32_t buf = tc & 1u;
         const uint32_t tph = (tc >> 1) & 1u;
+        const uint32_t idesc = decode_tile(sched, L, C::BN_OUT).rows <= 64 ? C::IDESC_M64 : C::IDESC;
         if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = sw128_desc(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = sw128_desc(b_addr + kk * 2048, CHUNK_BYTES, 1024);
-            umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued = true;
           umma_commit(&empty[s]);
@@ -289,7 +292,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;
     uint32_t tc = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tc) {
       const Tile t = decode_tile(sched, L, C::BN_OUT);
@@ -301,6 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // M = 64 accumulators hold tile row 16 q + i in lane i (< 16) of lane quarter q
+      const int r = t.rows <= 64 ? (lane < 16 ? q * 16 + lane : BM) : q * 32 + lane;
       const bool valid = r < t.rows;
       const uint32_t tacc = tmem_base + buf * kAccStride + ((uint32_t)(q * 32) << 16);
       if (MODE == kGateUp) {
