@@ -275,10 +275,13 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     // rows past the expert's end in its last K block first.
     constexpr bool kMN = MODE == kWG;
     constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kMN, kMN);
+    constexpr uint32_t IDESC_M64 = idesc_bf16_f32(64, BN, kMN, kMN);
     uint32_t it = 0, tc = 0;
     bool ok = true, issued = false;
     for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
       const Tile t = decode_tile<MODE>(sched, args, L);
+      // a row block of at most 64 rows (an expert's last) runs M = 64 MMAs
+      const uint32_t idesc = (MODE != kWG && t.rows <= 64) ? IDESC_M64 : IDESC;
       const uint32_t buf = tc & 1u;
       const uint32_t tph = (tc >> 1) & 1u;
       int got = 1;
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
               ad = sw128_desc(a_addr + kk * 32, 16, 1024);
               bd = sw128_desc(b_addr + kk * 32, 16, 1024);
             }
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued = true;
           umma_commit(&empty[s]);
@@ -362,7 +365,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;
     // column chunks of 32 this warp covers: all 8, or one half with 8 epilogue warps
     constexpr int kSplit = Warps<MODE>::kEpi / 4;
     const int half = kSplit == 1 ? 0 : (warp - 2) / 4;
@@ -379,6 +381,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * kAccStride + ((uint32_t)(q * 32) << 16);
+      // tile row of this thread; M = 64 accumulators hold row 16 q + i in lane i (< 16) of quarter q
+      const int r = (MODE != kWG && t.rows <= 64) ? (lane < 16 ? q * 16 + lane : BM) : q * 32 + lane;
       if (MODE == kDH) {
         const bool valid = r < t.rows;
         const int64_t row = t.m0 + r;
