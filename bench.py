@@ -569,6 +569,39 @@ def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, steps
     return res
 
 
+def graph_decode(moe, cfg, W, xs, out, ws, dev, stream, calls, eager_ms):
+    import torch
+
+    x_in = torch.empty_like(xs[0])
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        x_in.copy_(xs[0])
+        moe.layer_forward(cfg, x_in, W["wr"], W["wg"], W["wu"], W["wd"], out=out, ws=ws)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+        moe.layer_forward(cfg, x_in, W["wr"], W["wg"], W["wu"], W["wd"], out=out, ws=ws)
+    torch.cuda.synchronize(dev)
+    for i in range(3):
+        x_in.copy_(xs[i])
+        g.replay()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(calls):
+        x_in.copy_(xs[i])
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    return {"ms_per_call": ms / calls, "tokens_per_s": xs.shape[1] * calls / (ms / 1000.0),
+            "speedup_vs_eager": eager_ms / ms,
+            "note": "layer launches captured in one CUDA graph; each call = copy of x into the "
+                    "captured buffer + replay"}
+
+
 def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
     import torch
 
@@ -605,6 +638,12 @@ def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
            "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
            "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm",
            "kernel": "decode_gemm_kernel (weights on the MMA M side)"}
+    # the same calls replayed from a CUDA graph: the layer's launches are captured once
+    # and each call copies its x into the captured input buffer, then replays
+    try:
+        res["graph"] = graph_decode(moe, cfg, W, xs, out, ws, dev, stream, w.calls, ms)
+    except Exception as exc:  # capture is an optional measurement; report why it is missing
+        res["graph"] = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
     # the same calls with int8 expert weights (per-channel scales, int8 tensor cores)
     qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"])
     ws8 = torch.empty(moe.lib.moe_workspace_size_w8(cfg.ref), dtype=torch.uint8, device=dev)
