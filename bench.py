@@ -446,7 +446,9 @@ def main():
             "hbm_steps": hbm_steps(w, n_kept, per_kernel, fused, peaks),
             "path": ("down-combine fused: down sums into token order (its time includes the zeroing and "
                      "rounding passes; combine 0)") if fused else "separate down and combine",
-            "counts_kept": counts_kept, "n_kept": n_kept,
+            "counts_kept": counts_kept, "n_kept": n_kept, "dropped": 2 * w.T - n_kept,
+            "imbalance_max_over_mean_kept": max(counts_kept) / (sum(counts_kept) / len(counts_kept)),
+            "expert_utilization": [c * w.E / max(sum(counts_kept), 1) for c in counts_kept],
             "gpu_launches": launches_per_step * args.steps, "roofline": roofline, "clocks": clk}
 
     # ---- end to end: host x in, host out, through the C entry points with host buffers.

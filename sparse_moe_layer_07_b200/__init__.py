@@ -21,8 +21,10 @@ __all__ = [
     "MoEError", "Config", "LIB_PATH", "lib", "abi_version", "capacity", "workspace_size",
     "dispatch_workspace_size", "router_topk", "dispatch", "expert_ffn", "expert_gate_up",
     "expert_down", "combine", "layer_forward", "layer_forward_host", "get_device_error",
-    "STATUS", "DEVERR", "dispatch_noalloc", "NOALLOC_MAX_TOKENS", "quantize_int8", "expert_ffn_w8",
-    "layer_forward_w8", "QuantizedExperts", "w8_workspace_views",
+    "STATUS", "DEVERR", "ExpertUtilization", "dispatch_noalloc", "NOALLOC_MAX_TOKENS", "quantize_int8", "expert_ffn_w8",
+    "layer_forward_w8", "QuantizedExperts", "w8_workspace_views", "expert_down_combine",
+    "layer_forward_host_batches", "workspace_size_host_batches",
+    "workspace_size_train", "layer_forward_train", "layer_backward", "route_counts", "dispatch_shard", "gather_rows",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -505,6 +507,28 @@ def layer_forward_w8(cfg: Config, x, w_router, qw: QuantizedExperts, logit_bias=
                                     _dev_ptr(out), _dev_ptr(stats), _dev_ptr(ws), ws.numel(),
                                     _stream(stream, x.device)), "moe_layer_forward_w8")
     return out
+
+
+class ExpertUtilization:
+    """Router utilisation over many layer calls ("Training dynamics: expert
+    specialization": assignments per expert normalised so that a balanced
+    router gives 1.0 for every expert).  Feed it the stats array that
+    layer_forward fills (counts_raw in its first E entries); the running
+    counts stay on the device until utilization() is read."""
+
+    def __init__(self, E: int = 8, device="cuda"):
+        self.E = E
+        self.counts = torch.zeros(E, dtype=torch.int64, device=device)
+        self.calls = 0
+
+    def add(self, stats):
+        self.counts += stats[:self.E].to(torch.int64)
+        self.calls += 1
+
+    def utilization(self):
+        c = self.counts.double().cpu()
+        total = float(c.sum())
+        return (c * self.E / total).tolist() if total else [0.0] * self.E
 
 
 def get_device_error(clear: bool = True) -> int:

@@ -248,3 +248,23 @@ def test_bad_slot_in_combine_sets_device_error():
     assert moe.get_device_error(clear=True) & moe.DEVERR["SLOT_INDEX"]
     o = out.float().cpu()
     assert torch.all(o[0] == 1) and torch.all(o[1] == 0)
+
+
+def test_expert_utilization_over_calls():
+    # counts over several calls, normalised as the oracle's statistic (1.0 when balanced)
+    w = configs.scaled(W["grok_skew"], name="util", T=512, d=256, f=384)
+    L = LayerInputs(w)
+    D = L.dev
+    tracker = moe.ExpertUtilization()
+    idx_all = []
+    for call in range(4):
+        x = configs.make_x(w, call)
+        stats = torch.zeros(26, dtype=torch.int32, device="cuda")
+        moe.layer_forward(L.cfg, to_dev(x), D["wr"], D["wg"], D["wu"], D["wd"], logit_bias=D["bias"], stats=stats)
+        tracker.add(stats)
+        idx_all.append(oracle.top2_softmax(oracle.router_logits(x, L.wr, L.bias))[0])
+    torch.cuda.synchronize()
+    counts = np.bincount(np.concatenate(idx_all).ravel(), minlength=8)
+    want = oracle.expert_utilization(counts)
+    np.testing.assert_allclose(tracker.utilization(), want, rtol=0, atol=2 * 8 / counts.sum())
+    assert tracker.utilization()[0] > 1.5  # the biased expert
