@@ -161,6 +161,29 @@ def _check(status: int, where: str):
         raise MoEError(status, where)
 
 
+def _expect(name, t, numel, dtype):
+    """Host-side check of what the C ABI cannot see: element count and type."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name} must hold {numel} elements, got {t.numel()}")
+
+
+def _expect_layer(cfg, x=None, w_router=None, w_gate=None, w_up=None, w_down=None, logit_bias=None, out=None):
+    if cfg.T == 0:
+        return
+    dt = cfg.torch_dtype
+    _expect("x", x, cfg.T * cfg.d, dt)
+    _expect("w_router", w_router, cfg.E * cfg.d, dt)
+    _expect("w_gate", w_gate, cfg.E * cfg.d * cfg.f, dt)
+    _expect("w_up", w_up, cfg.E * cfg.d * cfg.f, dt)
+    _expect("w_down", w_down, cfg.E * cfg.f * cfg.d, dt)
+    _expect("logit_bias", logit_bias, cfg.E, torch.float32)
+    _expect("out", out, cfg.T * cfg.d, dt)
+
+
 def _empty(shape, dtype, like):
     return torch.empty(shape, dtype=dtype, device=like.device)
 
@@ -184,6 +207,7 @@ def dispatch_workspace_size(cfg: Config) -> int:
 def router_topk(cfg: Config, x, w_router, logit_bias=None, logits=None, topk_idx=None, topk_w=None,
                 want_logits: bool = False, stream=None):
     """Router logits, top-2 experts and their softmax weights.  Returns (idx, w, logits|None)."""
+    _expect_layer(cfg, x=x, w_router=w_router, logit_bias=logit_bias)
     if topk_idx is None:
         topk_idx = _empty((cfg.T, cfg.top_k), torch.int32, x)
     if topk_w is None:
@@ -350,6 +374,7 @@ def combine(cfg: Config, y, slot_of, topk_w=None, weights_applied: bool = True, 
 def layer_forward(cfg: Config, x, w_router, w_gate, w_up, w_down, logit_bias=None, out=None, stats=None,
                   ws=None, stream=None):
     """The whole layer; returns out [T, d] (stats, if given, is filled on the device)."""
+    _expect_layer(cfg, x, w_router, w_gate, w_up, w_down, logit_bias, out)
     if out is None:
         out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
     if ws is None:
@@ -365,6 +390,7 @@ def layer_forward_host(cfg: Config, x_host, w_router, w_gate, w_up, w_down, out_
     """The layer with x and out in (preferably pinned) host memory; returns when out_host is filled."""
     if x_host.is_cuda or out_host.is_cuda:
         raise ValueError("x_host and out_host must be host tensors")
+    _expect_layer(cfg, x_host, w_router, w_gate, w_up, w_down, logit_bias, out_host)
     _check(lib.moe_layer_forward_host(cfg.ref, _ptr(x_host), _dev_ptr(w_router), _dev_ptr(logit_bias),
                                       _dev_ptr(w_gate), _dev_ptr(w_up), _dev_ptr(w_down), _ptr(out_host),
                                       _dev_ptr(ws), ws.numel(), _stream(stream, w_router.device)),
@@ -387,6 +413,7 @@ def layer_forward_host_batches(cfg: Config, x_hosts, w_router, w_gate, w_up, w_d
     for t in list(x_hosts) + list(out_hosts):
         if t.dtype != cfg.torch_dtype or t.numel() != cfg.T * cfg.d:
             raise ValueError(f"host batches must be [T, d] = [{cfg.T}, {cfg.d}] of {cfg.dtype}")
+    _expect_layer(cfg, None, w_router, w_gate, w_up, w_down, logit_bias)
     n = len(x_hosts)
     xs = (ctypes.c_void_p * max(n, 1))(*[_ptr(t) for t in x_hosts])
     outs = (ctypes.c_void_p * max(n, 1))(*[_ptr(t) for t in out_hosts])
@@ -404,6 +431,7 @@ def workspace_size_train(cfg: Config) -> int:
 
 def layer_forward_train(cfg: Config, x, w_router, w_gate, w_up, w_down, ws, logit_bias=None, out=None, stream=None):
     """The layer forward that keeps the backward's inputs in ws (moe_workspace_size_train bytes)."""
+    _expect_layer(cfg, x, w_router, w_gate, w_up, w_down, logit_bias, out)
     if out is None:
         out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
     _check(lib.moe_layer_forward_train(cfg.ref, _dev_ptr(x), _dev_ptr(w_router), _dev_ptr(logit_bias),
@@ -416,6 +444,8 @@ def layer_backward(cfg: Config, x, w_router, w_gate, w_up, w_down, dout, ws, gra
                    stream=None):
     """Gradients of sum(out * dout) after layer_forward_train on the same ws.  Returns a dict of
     dx (layer dtype) and fp32 dw_router, dbias (or None), dw_gate, dw_up, dw_down."""
+    _expect_layer(cfg, x, w_router, w_gate, w_up, w_down)
+    _expect("dout", dout, cfg.T * cfg.d if cfg.T else dout.numel(), cfg.torch_dtype)
     E, d, f = cfg.E, cfg.d, cfg.f
     g = dict(grads or {})
     g.setdefault("dx", _empty((cfg.T, d), cfg.torch_dtype, x))
@@ -499,6 +529,7 @@ def expert_ffn_w8(cfg: Config, x_perm, offsets, qw: QuantizedExperts, row_scale=
 def layer_forward_w8(cfg: Config, x, w_router, qw: QuantizedExperts, logit_bias=None, out=None, stats=None, ws=None,
                      stream=None):
     """The whole layer with int8 expert weights; returns out [T, d]."""
+    _expect_layer(cfg, x=x, w_router=w_router, logit_bias=logit_bias, out=out)
     if out is None:
         out = _empty((cfg.T, cfg.d), cfg.torch_dtype, x)
     if ws is None:

@@ -219,3 +219,18 @@ def test_gather_rows_arguments_checked_before_launch(moe):
 def test_bounded_wait_check_limits(moe):
     assert moe.STATUS[moe.lib.moe_check_bounded_wait(10, None)] == "MOE_ERR_INVALID_ARG"
     assert moe.STATUS[moe.lib.moe_check_bounded_wait(2_000_000_000, None)] == "MOE_ERR_INVALID_ARG"
+
+
+def test_binding_checks_element_counts_and_types(moe):
+    import torch
+
+    c = _cfg(moe, T=4, d=128, f=128, dtype="bf16")
+    x = torch.zeros((4, 128), dtype=torch.float32)  # wrong type for a bf16 layer
+    wr = torch.zeros((8, 128), dtype=torch.bfloat16)
+    w = torch.zeros((8, 128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="x must be"):
+        moe.layer_forward(c, x, wr, w, w, w)
+    with pytest.raises(ValueError, match="w_gate must hold"):
+        moe.layer_forward(c, x.to(torch.bfloat16), wr, w[:4], w, w)
+    with pytest.raises(ValueError, match="logit_bias must be"):
+        moe.router_topk(c, x.to(torch.bfloat16), wr, logit_bias=torch.zeros(8, dtype=torch.float64))
