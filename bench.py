@@ -268,6 +268,8 @@ def main():
     ap.add_argument("--int8", action="store_true", help="int8 expert weights (weight-only, per-channel scales)")
     ap.add_argument("--no-train", action="store_true", help="skip the training pair (forward + backward)")
     ap.add_argument("--train-steps", type=int, default=5)
+    ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair"],
+                    help="tile shape of the bf16 grouped GEMMs (auto: CTA pairs at prefill sizes)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate down and combine kernels instead of the fused down-combine")
     args = ap.parse_args()
@@ -283,6 +285,7 @@ def main():
 
     import sparse_moe_layer_07_b200 as moe
 
+    moe.set_gemm_tiles(args.tiles)
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -405,6 +408,8 @@ def main():
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    # a pipeline wait that ran out of time sets the device error word: such a run is invalid
+    device_error = moe.get_device_error()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -444,6 +449,7 @@ def main():
             "tensor_frac_layer": tflops / peak,
             "kernels_ms": per_kernel,
             "hbm_steps": hbm_steps(w, n_kept, per_kernel, fused, peaks),
+            "gemm_tiles": args.tiles, "device_error": device_error,
             "path": ("down-combine fused: down sums into token order (its time includes the zeroing and "
                      "rounding passes; combine 0)") if fused else "separate down and combine",
             "counts_kept": counts_kept, "n_kept": n_kept, "dropped": 2 * w.T - n_kept,

@@ -377,6 +377,24 @@ MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void* x
  * with moe_get_device_error. */
 MOE_API moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t stream);
 
+/* Tile shape of the bf16 tensor-core grouped GEMMs (gate/up and down of the
+ * expert FFN, prefill sizes), a process-wide setting:
+ *   MOE_TILES_AUTO   the shape measured fastest on B200 (the default; single
+ *                    CTAs for every shape timed so far);
+ *   MOE_TILES_SINGLE one CTA per 128-row x N tile (M = 128 MMAs, M = 64 on an
+ *                    expert's last block of at most 64 rows);
+ *   MOE_TILES_PAIR   a cluster of two CTAs per 256-row tile (one 2-SM MMA of
+ *                    M = 256 spanning both SMs; an expert's last block is
+ *                    computed in full).
+ * Both shapes compute every output element with the same K-ordered fp32
+ * accumulation, so results do not depend on the mode.  Returns the previous
+ * mode in *previous (may be NULL); MOE_ERR_INVALID_ARG for an unknown mode.
+ * Calls already enqueued keep the shape they were launched with. */
+#define MOE_TILES_AUTO 0
+#define MOE_TILES_SINGLE 1
+#define MOE_TILES_PAIR 2
+MOE_API moe_status_t moe_set_gemm_tiles(int32_t mode, int32_t* previous);
+
 /* Waits for the current device, returns the device error word (MOE_DEVERR_*
  * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.
  * Returns MOE_ERR_DEVICE_CHECK when the word is non-zero, else MOE_OK. */

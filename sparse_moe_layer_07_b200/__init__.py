@@ -25,6 +25,7 @@ __all__ = [
     "layer_forward_w8", "QuantizedExperts", "w8_workspace_views", "expert_down_combine",
     "layer_forward_host_batches", "workspace_size_host_batches",
     "workspace_size_train", "layer_forward_train", "layer_backward", "route_counts", "dispatch_shard", "gather_rows",
+    "GEMM_TILES", "set_gemm_tiles", "gemm_tiles",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -88,6 +89,7 @@ def _load():
         "moe_expert_down_combine": ([cfgp, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_host_batches": ([cfgp, ctypes.c_int64, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32], ctypes.c_int),
+        "moe_set_gemm_tiles": ([ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
         "moe_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "moe_quantize_int8": ([cfgp, P, ctypes.c_int64, ctypes.c_int64, P, P, P], ctypes.c_int),
         "moe_expert_ffn_w8_workspace_size": ([cfgp], sz),
@@ -560,6 +562,38 @@ class ExpertUtilization:
         c = self.counts.double().cpu()
         total = float(c.sum())
         return (c * self.E / total).tolist() if total else [0.0] * self.E
+
+
+GEMM_TILES = {"auto": 0, "single": 1, "pair": 2}
+
+
+def set_gemm_tiles(mode: str) -> str:
+    """Tile shape of the bf16 grouped GEMMs for later calls (``moe_set_gemm_tiles``):
+    "auto", "single" (one CTA per 128-row tile) or "pair" (2-SM CTA pairs per
+    256-row tile).  Returns the previous mode."""
+    if mode not in GEMM_TILES:
+        raise ValueError(f"mode must be one of {sorted(GEMM_TILES)}")
+    prev = ctypes.c_int32(0)
+    st = lib.moe_set_gemm_tiles(GEMM_TILES[mode], ctypes.byref(prev))
+    if st != 0:
+        raise MoEError(st, "moe_set_gemm_tiles")
+    return {v: k for k, v in GEMM_TILES.items()}[prev.value]
+
+
+class gemm_tiles:
+    """Context manager: ``with gemm_tiles("pair"): ...`` restores the previous mode on exit."""
+
+    def __init__(self, mode: str):
+        self.mode = mode
+        self.prev = None
+
+    def __enter__(self):
+        self.prev = set_gemm_tiles(self.mode)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemm_tiles(self.prev)
+        return False
 
 
 def get_device_error(clear: bool = True) -> int:

@@ -65,6 +65,11 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
                            const void* wd, const float* row_scale, float* y, cudaStream_t s,
                            const Ctx& ctx);
 
+// Tile shape of the bf16 grouped GEMMs (MOE_TILES_*): one CTA per 128-row tile,
+// or CTA pairs (2-SM MMAs) per 256-row tile.  set_tile_mode returns the previous mode.
+int set_tile_mode(int mode);
+bool use_pair_tiles(const moe_config_t& c);
+
 // Down with the combine fused: adds row_scale * (H W_down) into a zeroed fp32
 // out32 [T, d] by token (perm) instead of writing Y.
 cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,

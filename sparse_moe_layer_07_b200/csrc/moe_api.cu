@@ -724,6 +724,13 @@ moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
   return cuda_status(launch_wait_check(limit_ns, stream, ctx));
 }
 
+moe_status_t moe_set_gemm_tiles(int32_t mode, int32_t* previous) {
+  if (mode != MOE_TILES_AUTO && mode != MOE_TILES_SINGLE && mode != MOE_TILES_PAIR) return MOE_ERR_INVALID_ARG;
+  const int prev = set_tile_mode(mode);
+  if (previous) *previous = prev;
+  return MOE_OK;
+}
+
 moe_status_t moe_get_device_error(int32_t* code, int32_t clear) {
   if (!code) return MOE_ERR_INVALID_ARG;
   Ctx ctx;
