@@ -221,6 +221,21 @@ def test_bounded_wait_check_limits(moe):
     assert moe.STATUS[moe.lib.moe_check_bounded_wait(2_000_000_000, None)] == "MOE_ERR_INVALID_ARG"
 
 
+def test_gemm_tile_mode_setting(moe):
+    import ctypes
+
+    prev = ctypes.c_int32(-1)
+    assert moe.STATUS[moe.lib.moe_set_gemm_tiles(7, ctypes.byref(prev))] == "MOE_ERR_INVALID_ARG"
+    assert prev.value == -1  # untouched on error
+    assert moe.set_gemm_tiles("pair") == "auto"
+    with moe.gemm_tiles("single"):
+        assert moe.set_gemm_tiles("single") == "single"
+    assert moe.set_gemm_tiles("auto") == "pair"  # the context manager restored "pair"
+    assert moe.STATUS[moe.lib.moe_set_gemm_tiles(0, None)] == "MOE_OK"
+    with pytest.raises(ValueError):
+        moe.set_gemm_tiles("quad")
+
+
 def test_binding_checks_element_counts_and_types(moe):
     import torch
 
