@@ -643,9 +643,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // cached per kernel.
 template <int MODE, bool FUSED>
 int pair_grid(const Ctx& ctx) {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];
   const int slot = ctx.dev >= 0 && ctx.dev < 64 ? ctx.dev : 0;
-  if (cached[slot] > 0) return cached[slot];
+  const int known = cached[slot].load(std::memory_order_relaxed);
+  if (known > 0) return known;
   auto kern = grouped_gemm_tc_pair_kernel<MODE, FUSED>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -664,7 +665,8 @@ int pair_grid(const Ctx& ctx) {
     n = ctx.num_sms / 2;
   }
   if (n > ctx.num_sms / 2) n = ctx.num_sms / 2;
-  cached[slot] = n;
+  if (n < 1) n = 1;
+  cached[slot].store(n, std::memory_order_relaxed);
   return n;
 }
 
