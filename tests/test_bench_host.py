@@ -74,3 +74,32 @@ def test_traffic_lookup_follows_the_kernel_sources(tmp_path, monkeypatch):
     assert bench.measured_traffic("mid_bf16") is None  # captured on the Grok prefill workload only
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(stale))
     assert bench.measured_traffic("grok_prefill") is None
+
+
+def test_clock_sampler_parses_and_filters_by_gpu(tmp_path, monkeypatch):
+    """A stand-in nvidia-smi on PATH prints samples of two GPUs; the sampler keeps
+    the named GPU's, takes the median SM clock and collects the active reasons."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text(
+        "#!/bin/sh\n"
+        "echo 'GPU-a, 1200, 1965, 900.5, Not Active, Not Active, Not Active, Active'\n"
+        "echo 'GPU-b, 300, 1965, 100.0, Active, Not Active, Not Active, Not Active'\n"
+        "echo 'GPU-a, 1300, 1965, 1001.0, Not Active, Not Active, Not Active, Active'\n"
+        "echo 'GPU-a, 1250, 1965, 950.0, Not Active, Not Active, Not Active, Not Active'\n"
+        "sleep 30\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
+    s = bench.ClockSampler("GPU-a")
+    s.start()
+    import time
+
+    for _ in range(100):
+        if len(s.rows) >= 3:
+            break
+        time.sleep(0.05)
+    r = s.stop()
+    assert r["samples"] == 3 and r["sm_mhz"] == 1250.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 1001.0
