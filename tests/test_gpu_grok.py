@@ -111,8 +111,10 @@ def test_grok_decode_full_size(grok):
 
 def test_grok_decode_int8_full_size(grok):
     """int8 expert weights at full Grok size: every code and scale against the
-    oracle's own quantisation, then the decode layer against the oracle's 8-bit
-    layer (its own codes for weights and rows)."""
+    oracle's own quantisation, then the decode layer against the weight-only
+    definition (the oracle's plain layer on exact activations and the
+    dequantised weights), and, as a check of the kernel's internals, against
+    the oracle's 8-bit layer that replays the activation row codes."""
     import sparse_moe_layer_07_b200 as moe
 
     host, dev = grok
@@ -141,11 +143,16 @@ def test_grok_decode_int8_full_size(grok):
         outs.append((L, g))
     # no capacity drop: tokens are independent, so one oracle call covers both batches
     x_all = np.concatenate([L.x for L, _ in outs])
-    ref = oracle.layer_forward_w8(x_all, host["wr"], *ref_q["wg"], *ref_q["wu"], *ref_q["wd"], float("inf"))
+    deq = [oracle.DequantizedExperts(*ref_q[k]) for k in ("wg", "wu", "wd")]
+    ref = oracle.layer_forward(x_all, host["wr"], *deq, float("inf"))
     res = [check_layer_out(L, g["out"], g["y"], g["slot_of"], ref["out"][i * w.T:(i + 1) * w.T], np.arange(w.T))
            for i, (L, g) in enumerate(outs)]
+    ref8 = oracle.layer_forward_w8(x_all, host["wr"], *ref_q["wg"], *ref_q["wu"], *ref_q["wd"], float("inf"))
+    res8 = [check_layer_out(L, g["out"], g["y"], g["slot_of"], ref8["out"][i * w.T:(i + 1) * w.T], np.arange(w.T))
+            for i, (L, g) in enumerate(outs)]
     REPORT["grok_decode_int8"] = {"calls_checked": list(calls), "weight_codes_bit_exact": True,
-                                  "max_err_over_rms": [list(r) for r in res]}
+                                  "max_err_over_rms_weight_only": [list(r) for r in res],
+                                  "max_err_over_rms_row_codes_replayed": [list(r) for r in res8]}
 
 
 def test_grok_train_full_size(grok):

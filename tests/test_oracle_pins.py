@@ -248,6 +248,27 @@ def pin_two_expert_dense(o):
     np.testing.assert_allclose(r["out"], w0[:, None] * y[0] + (1 - w0)[:, None] * y[1], rtol=1e-12, atol=1e-12)
 
 
+def pin_swiglu_expert_brute_force(o):
+    # one expert on its own (d != f, so a transposed operand cannot even run):
+    # swiglu_hidden and swiglu_expert against pure-Python loops, row by row
+    rng = np.random.default_rng(14)
+    n, d, f = 4, 5, 7
+    x = rng.standard_normal((n, d))
+    wg = rng.standard_normal((d, f)) / math.sqrt(d)
+    wu = rng.standard_normal((d, f)) / math.sqrt(d)
+    wd = rng.standard_normal((f, d)) / math.sqrt(f)
+    h = o.swiglu_hidden(x, wg, wu)
+    y = o.swiglu_expert(x, wg, wu, wd)
+    assert h.shape == (n, f) and y.shape == (n, d)
+    for r in range(n):
+        g = bf_matvec(x[r], wg.tolist())
+        u = bf_matvec(x[r], wu.tolist())
+        np.testing.assert_allclose(h[r], [gi / (1.0 + math.exp(-gi)) * ui for gi, ui in zip(g, u)],
+                                   rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(y[r], bf_expert(x[r], wg.tolist(), wu.tolist(), wd.tolist()),
+                                   rtol=1e-12, atol=1e-13)
+
+
 def pin_bf16_decoding(o):
     bits = np.array([0x3F80, 0xC000, 0x3E80, 0x0000, 0x8000, 0x4049], dtype=np.uint16)
     np.testing.assert_array_equal(o.to_f64(bits), [1.0, -2.0, 0.25, 0.0, -0.0, 3.140625])
@@ -468,7 +489,7 @@ ALL_PINS = [pin_router_logits, pin_top2_brute_force, pin_softmax_closed_form, pi
             pin_two_expert_dense, pin_bf16_decoding, pin_quantize_int8,
             pin_quantized_layer_uses_dequantized_weights, pin_quantize_rows, pin_int8_layer_exact,
             pin_backward_finite_differences, pin_backward_autograd, pin_backward_dropped_token,
-            pin_backward_subsets_and_slices]
+            pin_backward_subsets_and_slices, pin_swiglu_expert_brute_force]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -555,6 +576,7 @@ _orig_silu = O.silu
 _orig_router = O.router_logits
 _orig_hidden = O.swiglu_hidden
 _orig_capacity = O.capacity
+_orig_expert = O.swiglu_expert
 
 MUTANTS = {
     "silu_is_identity": dict(silu=lambda z: z),
@@ -566,6 +588,9 @@ MUTANTS = {
     "capacity_off_by_one": dict(dispatch=_dispatch_off_by_one),
     "capacity_floor": dict(capacity=lambda T, k, E, cf: T if math.isinf(cf) else int(math.floor(cf * T * k / E))),
     "gate_up_swapped": dict(swiglu_hidden=lambda x, g, u: _orig_hidden(x, u, g)),
+    "expert_gate_up_swapped": dict(swiglu_expert=lambda x, g, u, dn: _orig_expert(x, u, g, dn)),
+    "expert_silu_dropped": dict(swiglu_expert=lambda x, g, u, dn: ((O.to_f64(x) @ O.to_f64(g))
+                                                                   * (O.to_f64(x) @ O.to_f64(u))) @ O.to_f64(dn)),
     "quant_per_row": dict(quantize_int8=lambda w: _quant_rows(w)),
     "quant_scale_128": dict(quantize_int8=lambda w: _quant_div(w, 128.0)),
     "quant_floor": dict(quantize_int8=lambda w: _quant_floor(w)),
