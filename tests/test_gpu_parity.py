@@ -268,3 +268,24 @@ def test_expert_utilization_over_calls():
     want = oracle.expert_utilization(counts)
     np.testing.assert_allclose(tracker.utilization(), want, rtol=0, atol=2 * 8 / counts.sum())
     assert tracker.utilization()[0] > 1.5  # the biased expert
+
+
+def test_router_does_not_depend_on_the_batch():
+    """A token's logits, experts and weights are the same bits whatever batch it
+    arrives in: the router sums four fixed hidden-dimension quarters in a fixed
+    order, and only the number of CTAs sharing a tile changes with the batch
+    size (one, two or four here); also against the oracle's fp32 bound."""
+    w = configs.scaled(W["grok_skew"], name="router_batches", T=20000, d=512, f=256)
+    L = LayerInputs(w)
+    c = L.cfg
+    idx, wts, lg = moe.router_topk(c, L.dev["x"], L.dev["wr"], L.dev["bias"], want_logits=True)
+    g = {"idx": idx.cpu().numpy(), "w": wts.cpu().numpy(), "logits": lg.cpu().numpy().astype(np.float64)}
+    check_routing(L, g, oracle.router_logits(L.x, L.wr, L.bias))
+    for t0, n in ((0, 8192), (8192, 1000), (9192, 40), (19999, 1), (5000, 8000)):
+        cs = moe.Config(n, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16")
+        xs = L.dev["x"][t0:t0 + n].contiguous()
+        i2, w2, l2 = moe.router_topk(cs, xs, L.dev["wr"], L.dev["bias"], want_logits=True)
+        torch.cuda.synchronize()
+        assert torch.equal(l2, lg[t0:t0 + n]), (t0, n)
+        assert torch.equal(i2, idx[t0:t0 + n]) and torch.equal(w2, wts[t0:t0 + n]), (t0, n)
+    assert moe.get_device_error() == 0
