@@ -266,8 +266,11 @@ MOE_API size_t moe_workspace_size_host_batches(const moe_config_t* cfg);
  * copies to overlap.  Weights, logit_bias and ws are device memory; ws holds
  * moe_workspace_size_host_batches(cfg) bytes.  The work is ordered after the
  * work already in `stream`; the call returns when every out_host[i] is filled.
- * n_batches == 0 does nothing.  The two copy streams and their events are
- * created and destroyed inside the call (no device memory is allocated). */
+ * n_batches == 0 does nothing.  The two copy streams and their seven events
+ * are created on a device's first call and kept until the process exits
+ * (re-created after a context reset); no device memory is allocated.  Calls on
+ * one device from several host threads take turns (each call holds that
+ * device's copy streams until it returns). */
 MOE_API moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_batches,
                                             const void* const* x_host, const void* w_router,
                                             const float* logit_bias, const void* w_gate, const void* w_up,
@@ -363,8 +366,11 @@ MOE_API moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x
  * calls share that array: calls that overlap on the GPU (e.g. on two streams)
  * race.  The array keeps the last call's contents; each call writes every
  * entry it reads, so nothing needs clearing.  The first call on a device looks
- * up the array's device address with that device current; make it before any
- * stream capture.  No cudaMalloc, cudaFree or allocating routine is called. */
+ * up the array's device address with that device current and caches it for
+ * the current context; after cudaDeviceReset (a new context) the next call
+ * looks it up again.  Make the first call on a device, and the first after a
+ * reset, before any stream capture.  No cudaMalloc, cudaFree or allocating
+ * routine is called. */
 MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                                           const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
                                           int32_t* offsets, int32_t* perm, int32_t* slot_of,
@@ -394,6 +400,47 @@ MOE_API moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t strea
 #define MOE_TILES_SINGLE 1
 #define MOE_TILES_PAIR 2
 MOE_API moe_status_t moe_set_gemm_tiles(int32_t mode, int32_t* previous);
+
+/* Router utilisation over many calls ("How does Grok-1 use a
+ * mixture-of-experts design?", section "Training dynamics: expert
+ * specialization": assignments per expert normalised so that a balanced router
+ * gives 1.0 for every expert).  Adds stats[0..E) (the counts_raw a layer call
+ * wrote into its stats array) into the running int64 counts[E] and writes
+ * utilization[e] = counts[e] * E / sum(counts) (all 0 while the sum is 0),
+ * summed in expert order.  All three are device arrays owned by the caller;
+ * counts must start at zero for a new statistic.  1 <= E <= 64, else
+ * MOE_ERR_INVALID_ARG.  One small kernel on `stream`. */
+MOE_API moe_status_t moe_expert_utilization(const int32_t* stats, int32_t E, int64_t* counts, float* utilization,
+                                            moe_stream_t stream);
+
+/* Phase timing of the training pair, for measurement; the pages have no
+ * counterpart.  While enabled (moe_profile_phases(1), a process-wide setting),
+ * moe_layer_forward_train and moe_layer_backward record a pair of CUDA events
+ * on the call's stream around each of their kernels (events are created on
+ * first use and reused; nothing is recorded while disabled, the default).
+ * moe_profile_read waits for every recorded event, writes for each phase p < n
+ * the summed milliseconds ms[p] and the number of calls calls[p] since the
+ * previous read, and then forgets them.  ms and calls hold n entries (either
+ * may be NULL); n may be smaller than MOE_PHASE_COUNT.  At most 65536 event
+ * pairs are kept between reads; later ones are not recorded.  Returns
+ * MOE_ERR_CUDA if an event cannot be created or read. */
+#define MOE_PHASE_FWD_ROUTER 0   /* router logits + top-2 + softmax */
+#define MOE_PHASE_FWD_DISPATCH 1 /* histogram, scan, stable rank */
+#define MOE_PHASE_FWD_GATHER 2   /* x rows grouped by expert */
+#define MOE_PHASE_FWD_GATE_UP 3  /* gate/up + SwiGLU, G and U kept */
+#define MOE_PHASE_FWD_DOWN 4     /* down x routing weight */
+#define MOE_PHASE_FWD_COMBINE 5  /* weighted sum back to token order */
+#define MOE_PHASE_BWD_GATHER 6   /* dout by slot, routing-weighted copy */
+#define MOE_PHASE_BWD_DH 7       /* dH with the SwiGLU derivative -> dG, dU */
+#define MOE_PHASE_BWD_ZERO 8     /* fp32 dx accumulator cleared */
+#define MOE_PHASE_BWD_DX 9       /* dx = dG W_gate^T + dU W_up^T by token */
+#define MOE_PHASE_BWD_ROUTER 10  /* router backward, dx rounding */
+#define MOE_PHASE_BWD_WG_DOWN 11 /* dW_down */
+#define MOE_PHASE_BWD_WG_GATE 12 /* dW_gate */
+#define MOE_PHASE_BWD_WG_UP 13   /* dW_up */
+#define MOE_PHASE_COUNT 14
+MOE_API moe_status_t moe_profile_phases(int32_t enable);
+MOE_API moe_status_t moe_profile_read(float* ms, int32_t* calls, int32_t n);
 
 /* Waits for the current device, returns the device error word (MOE_DEVERR_*
  * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.

@@ -25,7 +25,7 @@ __all__ = [
     "layer_forward_w8", "QuantizedExperts", "w8_workspace_views", "expert_down_combine",
     "layer_forward_host_batches", "workspace_size_host_batches",
     "workspace_size_train", "layer_forward_train", "layer_backward", "route_counts", "dispatch_shard", "gather_rows",
-    "GEMM_TILES", "set_gemm_tiles", "gemm_tiles",
+    "GEMM_TILES", "set_gemm_tiles", "gemm_tiles", "PHASES", "profile_phases", "profile_read",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -96,6 +96,9 @@ def _load():
         "moe_workspace_size_w8": ([cfgp], sz),
         "moe_expert_ffn_w8": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_layer_forward_w8": ([cfgp, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_expert_utilization": ([P, ctypes.c_int32, P, P, P], ctypes.c_int),
+        "moe_profile_phases": ([ctypes.c_int32], ctypes.c_int),
+        "moe_profile_read": ([P, P, ctypes.c_int32], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         try:
@@ -552,16 +555,18 @@ class ExpertUtilization:
     def __init__(self, E: int = 8, device="cuda"):
         self.E = E
         self.counts = torch.zeros(E, dtype=torch.int64, device=device)
+        self.util = torch.zeros(E, dtype=torch.float32, device=device)
         self.calls = 0
 
-    def add(self, stats):
-        self.counts += stats[:self.E].to(torch.int64)
+    def add(self, stats, stream=None):
+        """moe_expert_utilization: counts += stats[:E] and the normalised statistic, on the device."""
+        _check(lib.moe_expert_utilization(_dev_ptr(stats), self.E, _dev_ptr(self.counts), _dev_ptr(self.util),
+                                          _stream(stream, stats.device)), "moe_expert_utilization")
         self.calls += 1
 
     def utilization(self):
-        c = self.counts.double().cpu()
-        total = float(c.sum())
-        return (c * self.E / total).tolist() if total else [0.0] * self.E
+        """The statistic after the last add() (a copy of the device array)."""
+        return self.util.cpu().tolist()
 
 
 GEMM_TILES = {"auto": 0, "single": 1, "pair": 2}
@@ -594,6 +599,24 @@ class gemm_tiles:
     def __exit__(self, *exc):
         set_gemm_tiles(self.prev)
         return False
+
+
+PHASES = ("fwd_router", "fwd_dispatch", "fwd_gather", "fwd_gate_up", "fwd_down", "fwd_combine",
+          "bwd_gather", "bwd_dh", "bwd_zero", "bwd_dx", "bwd_router", "bwd_wg_down", "bwd_wg_gate", "bwd_wg_up")
+
+
+def profile_phases(enable: bool) -> None:
+    """moe_profile_phases: record CUDA events around each kernel of the training pair."""
+    _check(lib.moe_profile_phases(int(bool(enable))), "moe_profile_phases")
+
+
+def profile_read() -> dict:
+    """moe_profile_read: {phase: (summed ms, calls)} since the previous read (waits for the events)."""
+    n = len(PHASES)
+    ms = (ctypes.c_float * n)()
+    calls = (ctypes.c_int32 * n)()
+    _check(lib.moe_profile_read(ms, calls, n), "moe_profile_read")
+    return {PHASES[i]: (float(ms[i]), int(calls[i])) for i in range(n)}
 
 
 def get_device_error(clear: bool = True) -> int:

@@ -313,4 +313,27 @@ cudaError_t launch_gather(const moe_config_t& c, const void* x, const int32_t* p
   return cudaGetLastError();
 }
 
+
+namespace {
+// counts[e] += stats[e]; utilization[e] = counts[e] * E / sum(counts), one
+// thread, experts in order (the sum does not depend on timing).
+__global__ void utilization_kernel(const int32_t* __restrict__ stats, int E, int64_t* __restrict__ counts,
+                                   float* __restrict__ util) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int64_t total = 0;
+  for (int e = 0; e < E; ++e) {
+    const int64_t c = counts[e] + (int64_t)stats[e];
+    counts[e] = c;
+    total += c;
+  }
+  for (int e = 0; e < E; ++e)
+    util[e] = total > 0 ? (float)((double)counts[e] * (double)E / (double)total) : 0.0f;
+}
+}  // namespace
+
+cudaError_t launch_utilization(const int32_t* stats, int E, int64_t* counts, float* util, cudaStream_t s) {
+  utilization_kernel<<<1, 32, 0, s>>>(stats, E, counts, util);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -5,16 +5,50 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe.h"
 
 namespace moe {
 
-// Per-device facts the launchers need.
+// NVTX range around an entry point (visible in Nsight timelines; no cost
+// without a tool attached).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
+
+// Phase timing (moe_profile_phases): while enabled, a PhaseMark records one
+// CUDA event on `s` when constructed and another at end(); the pair is kept
+// for moe_profile_read under MOE_PHASE_* index `phase`.  Disabled, it does
+// nothing.
+class PhaseMark {
+ public:
+  PhaseMark(int phase, cudaStream_t s);
+  void end();
+  ~PhaseMark() { end(); }
+  PhaseMark(const PhaseMark&) = delete;
+  PhaseMark& operator=(const PhaseMark&) = delete;
+
+ private:
+  int phase_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
+// Per-device facts the launchers need (looked up again when the device's
+// context changes, e.g. after cudaDeviceReset).
 struct Ctx {
   int dev = -1;
   int num_sms = 0;
   int* err = nullptr;  // device address of the device error word
+  unsigned long long ctx_id = 0;
 };
+
+// Unique id of the current CUDA context (cuCtxGetId); false when none is current.
+bool current_context_id(unsigned long long* id);
 
 // Rows of the grouped buffers (x_perm, h, y): every assignment may be kept.
 inline int64_t slot_rows(const moe_config_t& c) { return c.T * (int64_t)c.top_k; }
@@ -107,6 +141,9 @@ cudaError_t launch_round_out(const moe_config_t& c, const float* out32, void* ou
 // One block waits on an mbarrier nothing completes, bounded by limit_ns; sets
 // MOE_DEVERR_TIMEOUT when the wait gives up (check of the bounded-wait path).
 cudaError_t launch_wait_check(int64_t limit_ns, cudaStream_t s, const Ctx& ctx);
+
+// counts[e] += stats[e] and utilization[e] = counts[e] * E / sum(counts) (one block).
+cudaError_t launch_utilization(const int32_t* stats, int E, int64_t* counts, float* util, cudaStream_t s);
 
 // Argument check shared by the entry points (MOE_OK when the config is usable).
 moe_status_t validate_config(const moe_config_t* cfg);

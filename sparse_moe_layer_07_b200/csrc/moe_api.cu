@@ -25,19 +25,44 @@ constexpr int kMaxDevices = 64;
 Ctx g_ctx[kMaxDevices];
 std::mutex g_ctx_mu;
 
+// Driver entry points that identify the current context (resolved once).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fn_once;
+
+void resolve_ctx_fns() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+  p = nullptr;
+  if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(p);
+  (void)cudaGetLastError();
+}
+
+// Device facts of the current device, cached per device and context: the
+// symbol lookup also makes the device's primary context current if it was not.
 moe_status_t get_ctx(Ctx& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_ctx_mu);
   Ctx& c = g_ctx[dev];
-  if (c.dev != dev) {
+  unsigned long long id = 0;
+  if (c.dev != dev || !current_context_id(&id) || id != c.ctx_id) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_moe_device_error) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!current_context_id(&id)) return MOE_ERR_CUDA;
     c.num_sms = sms;
     c.err = static_cast<int*>(p);
     c.dev = dev;
+    c.ctx_id = id;
   }
   out = c;
   return MOE_OK;
@@ -156,6 +181,13 @@ moe_status_t run_down(const moe_config_t& c, const void* h, const int32_t* offse
 
 }  // namespace
 
+bool current_context_id(unsigned long long* id) {
+  std::call_once(g_ctx_fn_once, resolve_ctx_fns);
+  CUcontext c = nullptr;
+  return g_ctx_get_current && g_ctx_get_id && g_ctx_get_current(&c) == CUDA_SUCCESS && c != nullptr &&
+         g_ctx_get_id(c, id) == CUDA_SUCCESS;
+}
+
 moe_status_t validate_config(const moe_config_t* cfg) { return check_config(cfg); }
 
 moe_status_t current_ctx(Ctx& out) { return get_ctx(out); }
@@ -187,15 +219,6 @@ bool encode_tmap_dtype(CUtensorMap* map, const void* base, int rank, const uint6
 }  // namespace moe
 
 using namespace moe;
-
-namespace {
-// NVTX range around an entry point (visible in Nsight timelines; no cost
-// without a tool attached).
-struct Range {
-  explicit Range(const char* name) { nvtxRangePushA(name); }
-  ~Range() { nvtxRangePop(); }
-};
-}  // namespace
 
 extern "C" {
 
@@ -495,6 +518,52 @@ size_t moe_workspace_size_host_batches(const moe_config_t* cfg) {
   return layout_of(*cfg).total + 2 * round_up((size_t)cfg->T * cfg->d * esize(*cfg));
 }
 
+}  // extern "C"
+
+namespace moe {
+namespace {
+// The copy streams and events of moe_layer_forward_host_batches, created on a
+// device's first call and kept for the process (re-created when the device's
+// context changes, e.g. after cudaDeviceReset: the old handles died with it).
+// A call holds its device's lock from start to end (the call waits for its own
+// copies), so calls from several host threads on one device take turns.
+struct CopyPipe {
+  std::mutex mu;
+  bool ready = false;
+  unsigned long long ctx_id = 0;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev[7] = {};  // start, xin[2], comp[2], outfree[2]
+};
+CopyPipe g_pipes[kMaxDevices];
+
+// With the pipe's lock held: makes sure its streams and events exist in the current context.
+bool pipe_ready(CopyPipe& p, const Ctx& ctx) {
+  if (p.ready && p.ctx_id == ctx.ctx_id) return true;
+  p.ready = false;
+  p.h2d = p.d2h = nullptr;
+  for (cudaEvent_t& e : p.ev) e = nullptr;
+  bool ok = cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; ok && i < 7; ++i) ok = cudaEventCreateWithFlags(&p.ev[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    for (cudaEvent_t e : p.ev)
+      if (e) cudaEventDestroy(e);
+    if (p.h2d) cudaStreamDestroy(p.h2d);
+    if (p.d2h) cudaStreamDestroy(p.d2h);
+    p.h2d = p.d2h = nullptr;
+    for (cudaEvent_t& e : p.ev) e = nullptr;
+    (void)cudaGetLastError();
+    return false;
+  }
+  p.ctx_id = ctx.ctx_id;
+  p.ready = true;
+  return true;
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
 // Two-slot copy/compute pipeline: batch i uses staging slot i % 2 (x and out).
 //   h2d stream : wait comp[s] (batch i-2 done with slot s), copy x_host[i] -> x slot, record xin[s]
 //   stream     : wait xin[s] and outfree[s] (batch i-2's result copied out), layer, record comp[s]
@@ -524,14 +593,14 @@ moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_b
   uint8_t* x_slot[2] = {w8 + L.x_in, w8 + L.total};
   uint8_t* out_slot[2] = {w8 + L.out, w8 + L.total + round_up(bytes)};
 
-  cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t ev[7] = {};  // start, xin[2], comp[2], outfree[2]
+  CopyPipe& pipe = g_pipes[ctx.dev];
+  std::lock_guard<std::mutex> pipe_lock(pipe.mu);
+  if (!pipe_ready(pipe, ctx)) return MOE_ERR_CUDA;
+  cudaStream_t h2d = pipe.h2d, d2h = pipe.d2h;
+  cudaEvent_t* ev = pipe.ev;
   cudaEvent_t &start = ev[0], *xin = ev + 1, *comp = ev + 3, *outfree = ev + 5;
-  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
-  for (int i = 0; ok && i < 7; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
   // the whole pipeline starts after the work already in `stream`
-  ok = ok && cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(h2d, start, 0) == cudaSuccess &&
+  bool ok = cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(h2d, start, 0) == cudaSuccess &&
        cudaStreamWaitEvent(d2h, start, 0) == cudaSuccess;
   for (int64_t i = 0; ok && i < n_batches; ++i) {
     const int sl = (int)(i & 1);
@@ -549,14 +618,9 @@ moe_status_t moe_layer_forward_host_batches(const moe_config_t* cfg, int64_t n_b
   }
   // later work in `stream` is ordered after the last copy-out; then wait for all of it
   if (ok && st == MOE_OK) ok = cudaEventRecord(start, d2h) == cudaSuccess && cudaStreamWaitEvent(stream, start, 0) == cudaSuccess;
-  cudaError_t sync = cudaSuccess;
-  if (d2h) sync = cudaStreamSynchronize(d2h);
-  if (h2d && sync == cudaSuccess) sync = cudaStreamSynchronize(h2d);
+  cudaError_t sync = cudaStreamSynchronize(d2h);
+  if (sync == cudaSuccess) sync = cudaStreamSynchronize(h2d);
   if (sync == cudaSuccess) sync = cudaStreamSynchronize(stream);
-  for (int i = 0; i < 7; ++i)
-    if (ev[i]) cudaEventDestroy(ev[i]);
-  if (h2d) cudaStreamDestroy(h2d);
-  if (d2h) cudaStreamDestroy(d2h);
   if (st != MOE_OK) return st;
   if (!ok) return MOE_ERR_CUDA;
   return cuda_status(sync);
@@ -716,6 +780,16 @@ moe_status_t moe_layer_forward_w8(const moe_config_t* cfg, const void* x, const 
   return cuda_status(e);
 }
 
+moe_status_t moe_expert_utilization(const int32_t* stats, int32_t E, int64_t* counts, float* utilization,
+                                    moe_stream_t stream) {
+  Range range_("moe_expert_utilization");
+  if (!stats || !counts || !utilization || E < 1 || E > 64) return MOE_ERR_INVALID_ARG;
+  Ctx ctx;
+  moe_status_t st = get_ctx(ctx);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_utilization(stats, E, counts, utilization, stream));
+}
+
 moe_status_t moe_check_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
   if (limit_ns < 1000 || limit_ns > 1000000000) return MOE_ERR_INVALID_ARG;
   Ctx ctx;
@@ -823,16 +897,33 @@ moe_status_t moe_layer_forward_train(const moe_config_t* cfg, const void* x, con
   int32_t* slot_of = reinterpret_cast<int32_t*>(w8 + L.slot_of);
   float* row_scale = reinterpret_cast<float*>(w8 + L.row_scale);
   float* y = reinterpret_cast<float*>(w8 + L.y);
-  cudaError_t e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, stream, ctx);
-  if (e == cudaSuccess)
+  cudaError_t e;
+  {
+    PhaseMark m(MOE_PHASE_FWD_ROUTER, stream);
+    e = launch_router(c, x, w_router, logit_bias, nullptr, topk_idx, topk_w, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_FWD_DISPATCH, stream);
     e = launch_dispatch(c, capacity_of(c), topk_idx, topk_w, route, route + c.E, offsets, perm, slot_of, row_scale,
                         reinterpret_cast<int32_t*>(w8 + L.disp), nullptr, stream, ctx);
-  if (e == cudaSuccess) e = launch_gather(c, x, perm, offsets, w8 + L.x_perm, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_FWD_GATHER, stream);
+    e = launch_gather(c, x, perm, offsets, w8 + L.x_perm, stream, ctx);
+  }
   // the row-major tensor-core kernels at every batch size: gate/up keeps G and U
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_FWD_GATE_UP, stream);
     e = launch_tc_gate_up(c, w8 + L.x_perm, offsets, w_gate, w_up, w8 + L.h, stream, ctx, w8 + TL.g, w8 + TL.u);
-  if (e == cudaSuccess) e = launch_tc_down(c, w8 + L.h, offsets, w_down, row_scale, y, stream, ctx);
-  if (e == cudaSuccess) e = launch_combine(c, y, slot_of, topk_w, 1, out, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_FWD_DOWN, stream);
+    e = launch_tc_down(c, w8 + L.h, offsets, w_down, row_scale, y, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_FWD_COMBINE, stream);
+    e = launch_combine(c, y, slot_of, topk_w, 1, out, stream, ctx);
+  }
   return cuda_status(e);
 }
 
@@ -875,23 +966,43 @@ moe_status_t moe_layer_backward(const moe_config_t* cfg, const void* x, const vo
   float* dw_part = reinterpret_cast<float*>(w8 + TL.dw_part);
   float* dx32 = reinterpret_cast<float*>(w8 + TL.dx32);
   const int n_parts = (int)(c.f / 256) * bwd_dh_parts_per_tile();
-  cudaError_t e = launch_bwd_gather(c, dout, perm, offsets, row_scale, w8 + TL.dout_perm, w8 + TL.dy_perm, stream, ctx);
-  if (e == cudaSuccess)
+  cudaError_t e;
+  {
+    PhaseMark m(MOE_PHASE_BWD_GATHER, stream);
+    e = launch_bwd_gather(c, dout, perm, offsets, row_scale, w8 + TL.dout_perm, w8 + TL.dy_perm, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_DH, stream);
     e = launch_bwd_dh(c, w8 + TL.dout_perm, offsets, w_down, w8 + TL.g, w8 + TL.u, w8 + L.h, row_scale, w8 + TL.dg,
                       w8 + TL.du, dw_part, stream, ctx);
-  if (e == cudaSuccess) e = launch_zero_rows(c, dx32, stream, ctx);
-  if (e == cudaSuccess) e = launch_bwd_dx(c, w8 + TL.dg, w8 + TL.du, offsets, w_gate, w_up, perm, dx32, stream, ctx);
-  if (e == cudaSuccess)
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_ZERO, stream);
+    e = launch_zero_rows(c, dx32, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_DX, stream);
+    e = launch_bwd_dx(c, w8 + TL.dg, w8 + TL.du, offsets, w_gate, w_up, perm, dx32, stream, ctx);
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_ROUTER, stream);
     e = launch_router_bwd(c, dw_part, n_parts, slot_of, topk_idx, topk_w, w_router, dx32, x,
                           reinterpret_cast<float*>(w8 + TL.dlogits), reinterpret_cast<float*>(w8 + TL.dweight), dx,
                           dw_router, dbias, reinterpret_cast<float*>(w8 + TL.wr_part), stream, ctx);
+  }
   // weight gradients: the larger operand's blocks outermost, so the smaller one stays in L2
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_WG_DOWN, stream);
     e = launch_bwd_wgrad(c, w8 + L.h, c.f, w8 + TL.dy_perm, c.d, offsets, dw_down, c.f >= c.d, stream, ctx);
-  if (e == cudaSuccess)
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_WG_GATE, stream);
     e = launch_bwd_wgrad(c, w8 + L.x_perm, c.d, w8 + TL.dg, c.f, offsets, dw_gate, c.d >= c.f, stream, ctx);
-  if (e == cudaSuccess)
+  }
+  if (e == cudaSuccess) {
+    PhaseMark m(MOE_PHASE_BWD_WG_UP, stream);
     e = launch_bwd_wgrad(c, w8 + L.x_perm, c.d, w8 + TL.du, c.f, offsets, dw_up, c.d >= c.f, stream, ctx);
+  }
   return cuda_status(e);
 }
 
