@@ -19,8 +19,11 @@
 //   - the array keeps the last call's contents; nothing has to start at zero,
 //     because each call writes every histogram entry it later reads;
 //   - the first call on a device looks up the array's device address (with
-//     that device current) and caches it; make that first call before any
-//     stream capture.
+//     that device current) and caches it, keyed by the current context's
+//     unique id, so after a cudaDeviceReset (a new primary context) the next
+//     call looks the address up again; make the first call on a device, and
+//     the first after a reset, before any stream capture.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -40,19 +43,26 @@ static __device__ __align__(256) int32_t g_dispatch_scratch[kNoallocScratchInts]
 
 constexpr int kMaxDev = 64;
 int32_t* g_scratch_ptr[kMaxDev];
+unsigned long long g_scratch_ctx_id[kMaxDev];
 bool g_scratch_ready[kMaxDev];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch on the current device, looked up once per
-// device with that device current.
+// Device address of the scratch on the current device, looked up with that
+// device current the first time, and again whenever the current context is
+// not the one the cached address belongs to.
 moe_status_t scratch_on_current_device(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ready[dev]) {
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (!g_scratch_ready[dev] || !have_id || id != g_scratch_ctx_id[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    // the lookup makes the device's primary context current if it was not yet
+    if (!current_context_id(&id)) return MOE_ERR_CUDA;
     g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    g_scratch_ctx_id[dev] = id;
     g_scratch_ready[dev] = true;
   }
   *out = g_scratch_ptr[dev];
@@ -70,6 +80,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
                                              const float* topk_w, int32_t* counts_raw, int32_t* counts_kept,
                                              int32_t* offsets, int32_t* perm, int32_t* slot_of, float* row_scale,
                                              void* x_perm, moe_stream_t stream) {
+  Range range_("moe_dispatch_noalloc");
   moe_status_t st = validate_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T > MOE_NOALLOC_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;

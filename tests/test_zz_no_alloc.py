@@ -43,3 +43,26 @@ def test_noalloc_dispatch_matches_dispatch(T, call):
     assert torch.equal(got["row_scale"][:n], ref["row_scale"][:n])
     assert torch.equal(got["x_perm"][:n], ref["x_perm"][:n])
     assert moe.get_device_error() == 0
+
+
+def test_noalloc_dispatch_at_the_size_limit():
+    # T = MOE_NOALLOC_MAX_TOKENS: the last histogram block's entries reach the end
+    # of the fixed array; one more token is refused before any launch
+    T, d = moe.NOALLOC_MAX_TOKENS, 128
+    x = torch.from_numpy(configs.normal(configs.SEED, 950, (T, d), dtype="bf16")).view(torch.bfloat16).cuda()
+    wr = torch.from_numpy(configs.normal(configs.SEED, 951, (8, d), std=0.02, dtype="bf16")).view(torch.bfloat16)
+    cfg = moe.Config(T, d, 128, capacity_factor=1.0, dtype="bf16")
+    idx, wts, _ = moe.router_topk(cfg, x, wr.cuda())
+    ref = moe.dispatch(cfg, x, idx, wts, gather=False)
+    got = moe.dispatch_noalloc(cfg, x, idx, wts, gather=False)
+    torch.cuda.synchronize()
+    for k in ("counts_raw", "counts_kept", "offsets", "slot_of"):
+        assert torch.equal(got[k], ref[k]), k
+    n = int(ref["offsets"][-1])
+    assert int(ref["counts_raw"].sum()) == 2 * T and n < 2 * T  # cf 1.0: the fuller experts drop some
+    assert torch.equal(got["perm"][:n], ref["perm"][:n])
+    assert torch.equal(got["row_scale"][:n], ref["row_scale"][:n])
+    assert moe.get_device_error() == 0
+    big = moe.Config(T + 1, d, 128, capacity_factor=1.0, dtype="bf16")
+    with pytest.raises(RuntimeError, match="MOE_ERR_UNSUPPORTED"):
+        moe.dispatch_noalloc(big, x, idx, wts, gather=False)
