@@ -9,7 +9,10 @@ C ABI.  Prints one JSON line on rank 0.
 Workload default: the Grok-1-shape prefill layer (T=8192, d=6144, f=32768,
 E=8, top-2, no drop).  Under torchrun every rank runs its own batch (distinct
 x, same weights): the layer shards by token batch with no collective on the
-data path ("weak" scaling); timing is the max over ranks.
+data path ("weak" scaling); timing is the max over ranks.  On one GPU the line
+also carries a per-configuration block (the mid bf16 layer, the skewed Grok
+layer, the Grok decode calls and the tiny fp32 layer), each entry timed with
+its own clock record.
 """
 from __future__ import annotations
 
@@ -30,7 +33,10 @@ sys.path.insert(0, ROOT)
 
 from synth import configs  # noqa: E402
 
-PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the pool's earlier measurement: burst cuBLAS bf16, and the sustained figure with
+# the SM clock it settled at under the power cap
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "bf16_tflops_sustained_sm_mhz": 1300.0}
 
 
 def load_peaks():
@@ -42,35 +48,83 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_tc_dram_grok_prefill_T8192_d6144_f32768.md")
-KERNEL_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_07_b200", "csrc", n) for n in ("ffn_tc.cu", "tc_ptx.cuh")]
+def _num(v):
+    try:
+        return float(v)
+    except (TypeError, ValueError):
+        return None
 
 
-def measured_traffic(workload_name):
-    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary,
-    or None when the workload differs or the kernel sources changed since the capture."""
+def _sustained_clock_mhz(peaks):
+    """SM clock (MHz) at which the sustained tensor peak was measured, when recorded:
+    a key of its own, or the median of the clock record taken under load."""
+    for key in ("bf16_tflops_sustained_sm_mhz", "bf16_tflops_sustained_clock_mhz"):
+        if _num(peaks.get(key)):
+            return _num(peaks[key])
+    sect = peaks.get("clocks_under_load")
+    if _num(sect):
+        return _num(sect)
+    if isinstance(sect, dict):
+        for key in ("sm_mhz_median", "median_sm_mhz", "sm_mhz", "median", "clocks.sm"):
+            if _num(sect.get(key)):
+                return _num(sect[key])
+    return None
+
+
+def tensor_peak(peaks, src, clk):
+    """The dense bf16 tensor peak that matches the clock the run actually had.
+
+    The burst figure (a GEMM timed alone, at full clock) applies when the run's
+    median SM clock is within 5% of the maximum.  Below that the run was held
+    down by the power cap: the sustained figure is scaled by (the run's median
+    SM MHz / the MHz it was measured at), and never taken above the burst
+    figure; without a record of that clock the sustained figure is used as it
+    is.  Returns (peak TFLOP/s, the rule used)."""
+    burst = _num(peaks.get("bf16_tflops")) or PEAKS_FALLBACK["bf16_tflops"]
+    sm = _num((clk or {}).get("sm_mhz"))
+    smax = _num((clk or {}).get("sm_max_mhz"))
+    if sm and smax and sm >= 0.95 * smax:
+        return burst, f"{src} bf16_tflops (burst): run median SM clock {sm:.0f} MHz within 5% of max {smax:.0f}"
+    sus = _num(peaks.get("bf16_tflops_sustained"))
+    at = _sustained_clock_mhz(peaks)
+    if sm and sus and at:
+        p = min(burst, sus * sm / at)
+        return p, (f"{src} bf16_tflops_sustained x run median SM clock {sm:.0f} MHz / {at:.0f} MHz at which it "
+                   f"was measured (capped at the burst figure)")
+    if sus:
+        return sus, f"{src} bf16_tflops_sustained: run SM clock below 95% of max or not recorded"
+    return burst, f"{src} bf16_tflops (burst): no clock record"
+
+
+# DRAM traffic per launch of the roofline kernel, from a committed ncu capture
+# (machine-readable; the summary beside it in profiles/ gives the command).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_07_b200", "csrc", n)
+                  for n in ("ffn_tc.cu", "tc_ptx.cuh", "common.cuh", "internal.h")]
+
+
+def kernel_sources_sha256():
     import hashlib
 
-    if workload_name != "grok_prefill" or not os.path.exists(TRAFFIC_FILE):
-        return None
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
         with open(p, "rb") as fh:
             h.update(fh.read())
-    fields = {}
+    return h.hexdigest()
+
+
+def measured_traffic(workload_name, kernel="gate_up"):
+    """DRAM read + write bytes per launch of `kernel` on this workload from the
+    committed capture, or None when there is none or the kernel sources changed
+    since it was taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
     with open(TRAFFIC_FILE) as fh:
-        for line in fh:
-            if ":" in line:
-                k, v = line.strip().split(":", 1)
-                fields[k.strip()] = v.strip()
-    if fields.get("kernel_sources_sha256") != h.hexdigest():
+        d = json.load(fh)
+    if d.get("kernel_sources_sha256") != kernel_sources_sha256():
         return None
-    try:
-        return float(fields["gate_up_dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
-
-
+    entry = d.get("workloads", {}).get(workload_name, {}).get(kernel)
+    return _num(entry.get("dram_bytes_per_launch")) if isinstance(entry, dict) else None
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -127,6 +181,7 @@ class ClockSampler:
     def __init__(self, uuid: str):
         self.uuid = uuid
         self.rows = []
+        self.times = []
         self.proc = None
         self.thread = None
 
@@ -145,8 +200,11 @@ class ClockSampler:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) == 8 and (not self.uuid or parts[0] == self.uuid):
                 self.rows.append(parts)
+                self.times.append(time.monotonic())
 
-    def stop(self):
+    def stop(self, window=None):
+        """Stops sampling; `window` = (t0, t1) in time.monotonic() keeps the
+        samples taken inside it (the nearest later one when none falls inside)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -156,6 +214,13 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
+        if window is not None and self.rows:
+            t0, t1 = window
+            keep = [r for r, t in zip(self.rows, self.times) if t0 <= t <= t1 + 0.15]
+            if not keep:
+                later = [r for r, t in zip(self.rows, self.times) if t >= t0]
+                keep = later[:1]
+            self.rows = keep
         sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -176,16 +241,66 @@ def blas_threads():
         return 1
 
 
-def oracle_sample(w, host, x, n_tokens, seed):
-    """Time the oracle on a seeded token sample of this workload (routing over all T)."""
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_layer_time(w, host, x, n_sample, seed, threads=None):
+    """The oracle's time for the whole layer, by the recipe of the measurement plan:
+    router, top-2 and dispatch timed over all T tokens; the expert FFN and the
+    combine timed on a seeded sample of tokens and extrapolated per kept
+    assignment (x N_kept / kept assignments in the sample).  `threads` limits
+    the BLAS threads (None: the library's default, all cores)."""
+    import contextlib
+
     import oracle
 
+    limit = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+
+        limit = threadpool_limits(limits=threads, user_api="blas")
     rng = np.random.default_rng(seed)
-    tok = np.sort(rng.choice(w.T, size=min(n_tokens, w.T), replace=False))
-    t0 = time.perf_counter()
-    oracle.layer_forward(x, host["wr"], host["wg"], host["wu"], host["wd"], w.capacity_factor,
-                         logit_bias=configs.make_bias(w), tokens=tok)
-    return time.perf_counter() - t0, len(tok)
+    tok = np.sort(rng.choice(w.T, size=min(n_sample, w.T), replace=False))
+    bias = configs.make_bias(w)
+    with limit:
+        used = blas_threads()
+        t0 = time.perf_counter()
+        lg = oracle.router_logits(x, host["wr"], bias)
+        idx, wt = oracle.top2_softmax(lg)
+        disp = oracle.dispatch(idx, wt, w.E, oracle.capacity(w.T, w.top_k, w.E, w.capacity_factor))
+        t_route = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.layer_forward(x, host["wr"], host["wg"], host["wu"], host["wd"], w.capacity_factor, logit_bias=bias,
+                             tokens=tok)
+        t_sample = time.perf_counter() - t0
+    # layer_forward routes all T again before the sampled FFN: that share is t_route
+    t_ffn = max(t_sample - t_route, 0.0)
+    kept_sample = int((disp["slot_of"][tok] >= 0).sum())
+    n_kept = int(disp["n_kept"])
+    scale = n_kept / kept_sample if kept_sample else 0.0
+    t_layer = t_route + t_ffn * scale
+    return {"layer_s": t_layer, "tokens_per_s": w.T / t_layer, "route_s": t_route, "ffn_sample_s": t_ffn,
+            "sample_tokens": int(tok.size), "kept_in_sample": kept_sample, "n_kept": n_kept,
+            "extrapolation": scale, "threads": used}
+
+
+def cpu_baseline(w, host, x, n_sample):
+    """The oracle on this host's cores, single-threaded and on all cores."""
+    one = oracle_layer_time(w, host, x, n_sample, 7, threads=1)
+    allc = oracle_layer_time(w, host, x, n_sample, 7)
+    return {"value": allc["tokens_per_s"], "unit": "tokens/s", "cores": allc["threads"], "kind": "oracle",
+            "nproc": host_cores(),
+            "sample": (f"oracle (fp64 numpy): router, top-2 and dispatch over all T={w.T} tokens "
+                       f"({allc['route_s']:.2f} s); expert FFN and combine on {allc['sample_tokens']} seeded tokens "
+                       f"({allc['kept_in_sample']} kept assignments, {allc['ffn_sample_s']:.2f} s) extrapolated "
+                       f"x{allc['extrapolation']:.1f} to the {allc['n_kept']} kept assignments of the layer"),
+            "layer_s": allc["layer_s"],
+            "single_thread": {"value": one["tokens_per_s"], "cores": one["threads"], "layer_s": one["layer_s"],
+                              "route_s": one["route_s"], "ffn_sample_s": one["ffn_sample_s"]}}
 
 
 def reference_arm(args, w):
@@ -195,31 +310,40 @@ def reference_arm(args, w):
     host = dict(wr=configs.make_router(w), wg=configs.make_w_gate(w), wu=configs.make_w_up(w),
                 wd=configs.make_w_down(w))
     x = configs.make_x(w)
-    per_step = args.ref_tokens
+    n = args.ref_tokens
+    # Each step is one oracle measurement of the whole layer (routing over all T,
+    # the FFN on an n-token sample extrapolated per kept assignment); steps stop
+    # once the next one would pass the wall-clock budget, so a long --steps
+    # still ends within a few minutes.  Warm-up steps stop at a third of it.
+    t_w, warm = 0.0, 0
     for i in range(args.warmup):
-        oracle_sample(w, host, x, per_step, 1000 + i)
-    # Each step is a few seconds of fp64 work on the host (the expert matrices of the
-    # sampled tokens are widened to fp64 per call); steps stop once the next one would
-    # pass the wall-clock budget, so a long --steps still ends within a few minutes.
-    tot, ntok, done = 0.0, 0, 0
-    for i in range(args.steps):
-        if done and tot + tot / done > args.ref_budget_s:
+        if warm and t_w + t_w / warm > args.ref_budget_s / 3:
             break
-        t, n = oracle_sample(w, host, x, per_step, i)
-        tot += t
-        ntok += n
+        t0 = time.perf_counter()
+        oracle_layer_time(w, host, x, n, 1000 + i)
+        t_w += time.perf_counter() - t0
+        warm += 1
+    layer_s, wall, done, r = [], 0.0, 0, None
+    for i in range(args.steps):
+        if done and wall + wall / done > args.ref_budget_s:
+            break
+        t0 = time.perf_counter()
+        r = oracle_layer_time(w, host, x, n, i)
+        wall += time.perf_counter() - t0
+        layer_s.append(r["layer_s"])
         done += 1
-    value = ntok / tot
-    cores = blas_threads()
-    sample = (f"oracle (fp64 numpy) per step: router, top-2 and dispatch over all T={w.T} tokens, "
-              f"expert FFN and combine for {per_step} seeded tokens; {done} of {args.steps} requested steps "
-              f"timed (wall-clock budget {args.ref_budget_s:.0f} s)")
+    ms = 1000.0 * statistics.fmean(layer_s)
+    value = w.T / (ms / 1000.0)
+    sample = (f"oracle (fp64 numpy) per step: router, top-2 and dispatch over all T={w.T} tokens, expert FFN and "
+              f"combine on {n} seeded tokens extrapolated per kept assignment to the whole layer; {done} of "
+              f"{args.steps} requested steps timed (wall-clock budget {args.ref_budget_s:.0f} s), {warm} warm-up")
     line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": done, "steps_requested": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000 * tot / done, "higher_is_better": True, "scaling": "weak",
+            "n_gpus": args.gpus, "steps": done, "steps_requested": args.steps, "warmup": warm,
+            "warmup_requested": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["threads"], "nproc": host_cores(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -251,6 +375,160 @@ def workload_config(w):
 
 
 # ---------------------------------------------------------------------------- our arm
+class LayerRun:
+    """Device buffers of one workload and one step of the layer through the
+    separate entry points (router -> dispatch -> gate/up -> down + combine),
+    with CUDA events between the calls."""
+
+    NAMES = ["router", "dispatch", "gate_up", "down", "combine"]
+
+    def __init__(self, moe, w, W, x, bias_d, dev, stream, int8=False, unfused=False):
+        import torch
+
+        self.moe, self.w, self.W, self.x, self.bias_d, self.dev, self.stream = moe, w, W, x, bias_d, dev, stream
+        self.cfg = cfg = moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype=w.storage)
+        rows = w.T * w.top_k
+        tdt = cfg.torch_dtype
+        self.buf = {
+            "idx": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
+            "w": torch.empty((w.T, 2), dtype=torch.float32, device=dev),
+            "h": torch.empty((rows, w.f), dtype=tdt, device=dev),
+            "out": torch.empty((w.T, w.d), dtype=tdt, device=dev),
+            "ws": torch.empty((max(moe.dispatch_workspace_size(cfg), 16),), dtype=torch.uint8, device=dev),
+        }
+        self.disp = {"counts_raw": torch.empty(8, dtype=torch.int32, device=dev),
+                     "counts_kept": torch.empty(8, dtype=torch.int32, device=dev),
+                     "offsets": torch.empty(9, dtype=torch.int32, device=dev),
+                     "perm": torch.empty(rows, dtype=torch.int32, device=dev),
+                     "slot_of": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
+                     "row_scale": torch.empty(rows, dtype=torch.float32, device=dev),
+                     "x_perm": torch.empty((rows, w.d), dtype=tdt, device=dev)}
+        self.qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"]) if int8 else None
+        self.ws8 = (torch.empty((max(moe.lib.moe_expert_ffn_w8_workspace_size(cfg.ref), 16),), dtype=torch.uint8,
+                                device=dev) if int8 else None)
+        # bf16 tensor-core batches sum the down outputs into token order (zero + down
+        # + rounding pass, no y buffer, no separate combine)
+        self.fused = (not int8 and not unfused and w.storage == "bf16" and w.T * 2 > 64 * w.E and w.d % 256 == 0)
+        if self.fused:
+            self.buf["dc_ws"] = torch.empty(moe.lib.moe_expert_down_combine_workspace_size(cfg.ref),
+                                            dtype=torch.uint8, device=dev)
+        else:
+            self.buf["y"] = torch.empty((rows, w.d), dtype=torch.float32, device=dev)
+        # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code
+        # passes and the partial sum); fused: router 1, dispatch 3 + gather 1, gate/up 1, zero + down +
+        # rounding 3
+        self.launches_per_step = 11 if int8 else (9 if self.fused else 8)
+
+    def step(self, ev=None):
+        moe, cfg, W, buf, disp, s = self.moe, self.cfg, self.W, self.buf, self.disp, self.stream
+
+        def mark(i):
+            if ev:
+                ev[i].record(s)
+
+        mark(0)
+        moe.router_topk(cfg, self.x, W["wr"], self.bias_d, topk_idx=buf["idx"], topk_w=buf["w"])
+        mark(1)
+        moe.dispatch(cfg, self.x, buf["idx"], buf["w"], out=disp, ws=buf["ws"])
+        mark(2)
+        if self.qw is not None:
+            # int8 experts: gate/up and down in one call (both timed under "gate_up")
+            moe.expert_ffn_w8(cfg, disp["x_perm"], disp["offsets"], self.qw, disp["row_scale"], y=buf["y"],
+                              ws=self.ws8)
+        else:
+            moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
+        mark(3)
+        if self.fused:
+            moe.expert_down_combine(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], disp["perm"],
+                                    out=buf["out"], ws=buf["dc_ws"])
+            mark(4)
+            mark(5)
+            return
+        if self.qw is None:
+            moe.expert_down(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], y=buf["y"])
+        mark(4)
+        moe.combine(cfg, buf["y"], disp["slot_of"], buf["w"], weights_applied=True, out=buf["out"])
+        mark(5)
+
+    def time(self, steps, warmup, world=1):
+        """W untimed steps, then K steps between a barrier + synchronize on both
+        sides, clocks sampled during the timed region; the max over ranks."""
+        import torch
+        import torch.distributed as dist
+
+        dev, stream = self.dev, self.stream
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize(dev)
+        n_kept = int(self.disp["offsets"][-1].item())
+        counts_kept = self.disp["counts_kept"].cpu().tolist()
+        counts_raw = self.disp["counts_raw"].cpu().tolist()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        uuid = ""
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:
+            pass
+        clocks = ClockSampler(uuid)
+        clocks.start()
+        time.sleep(0.5)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        w0 = time.monotonic()
+        t_start.record(stream)
+        for i in range(steps):
+            self.step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        w1 = time.monotonic()
+        # a pipeline wait that ran out of time sets the device error word: such a run is invalid
+        device_error = self.moe.get_device_error()
+        if world > 1:
+            dist.barrier()
+        clk = clocks.stop(window=(w0, w1))
+        ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev, world)
+        per_kernel = {n: 0.0 for n in self.NAMES}
+        for e in evs:
+            for j, n in enumerate(self.NAMES):
+                per_kernel[n] += e[j].elapsed_time(e[j + 1])
+        per_kernel = {n: v / steps for n, v in per_kernel.items()}
+        return {"ms_total": ms_total, "ms_step": ms_total / steps, "per_kernel": per_kernel, "n_kept": n_kept,
+                "counts_kept": counts_kept, "counts_raw": counts_raw, "device_error": device_error, "clocks": clk}
+
+
+def gemm_roofline(w, res, peaks, src):
+    """Achieved TFLOP/s of the gate/up and down kernels against the clock-matched tensor peak."""
+    n = res["n_kept"]
+    pk = res["per_kernel"]
+    peak, rule = tensor_peak(peaks, src, res["clocks"])
+    gu = 4.0 * n * w.d * w.f / (pk["gate_up"] / 1000.0) / 1e12 if pk["gate_up"] > 0 else 0.0
+    dn = 2.0 * n * w.d * w.f / (pk["down"] / 1000.0) / 1e12 if pk["down"] > 0 else 0.0
+    return peak, rule, gu, dn
+
+
+def layer_summary(w, res, peaks, src, world, steps):
+    """tokens/s, TFLOP/s, GEMM roofline fractions, drops and balance of one timed workload."""
+    n = res["n_kept"]
+    ms = res["ms_total"]
+    flops_step = 2.0 * w.T * w.d * w.E + 6.0 * n * w.d * w.f
+    peak, rule, gu, dn = gemm_roofline(w, res, peaks, src)
+    ck = res["counts_kept"]
+    tf = world * flops_step * steps / (ms / 1000.0) / 1e12
+    return {"workload": w.name, "T": w.T, "d": w.d, "f": w.f, "capacity_factor": w.capacity_factor,
+            "dtype": "bf16" if w.storage == "bf16" else "f32",
+            "tokens_per_s": throughput(world, w.T, steps, ms), "ms_per_step": res["ms_step"], "steps": steps,
+            "tflops": tf, "tensor_frac_layer": tf / peak,
+            "gate_up": {"tflops": gu, "frac": gu / peak}, "down": {"tflops": dn, "frac": dn / peak},
+            "peak_tflops": peak, "peak_rule": rule, "kernels_ms": res["per_kernel"],
+            "n_kept": n, "dropped": w.top_k * w.T - n, "counts_raw": res["counts_raw"], "counts_kept": ck,
+            "expert0_share_raw": res["counts_raw"][0] / max(sum(res["counts_raw"]), 1),
+            "imbalance_max_over_mean_kept": max(ck) / (sum(ck) / len(ck)) if sum(ck) else None,
+            "device_error": res["device_error"], "clocks": res["clocks"]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -258,18 +536,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="grok_prefill", choices=sorted(configs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per reference-arm step")
+    ap.add_argument("--ref-tokens", type=int, default=64, help="sampled tokens per reference-arm step")
     ap.add_argument("--ref-budget-s", type=float, default=150.0, help="wall-clock budget of the reference arm's steps")
     ap.add_argument("--cpu-tokens", type=int, default=64, help="tokens in the CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration block")
     ap.add_argument("--shape", default=None, help="T,d,f override of the workload (profiling cases)")
     ap.add_argument("--int8", action="store_true", help="int8 expert weights (weight-only, per-channel scales)")
     ap.add_argument("--no-train", action="store_true", help="skip the training pair (forward + backward)")
     ap.add_argument("--train-steps", type=int, default=5)
     ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair"],
-                    help="tile shape of the bf16 grouped GEMMs (auto: CTA pairs at prefill sizes)")
+                    help="tile shape of the bf16 grouped GEMMs")
     ap.add_argument("--unfused", action="store_true",
                     help="separate down and combine kernels instead of the fused down-combine")
     args = ap.parse_args()
@@ -294,16 +573,12 @@ def main():
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
-    def to_dev(a):
-        t = torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-        return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
-
     # ---- inputs: weights generated once (rank 0) and broadcast; x distinct per rank
     host = None
     if rank == 0:
         host = dict(wr=configs.make_router(w), wg=configs.make_w_gate(w), wu=configs.make_w_up(w),
                     wd=configs.make_w_down(w))
-        W = {k: to_dev(v) for k, v in host.items()}
+        W = {k: to_dev(v, dev) for k, v in host.items()}
     else:
         tdt = torch.bfloat16 if w.storage == "bf16" else torch.float32
         W = {"wr": torch.empty((w.E, w.d), dtype=tdt, device=dev),
@@ -312,224 +587,173 @@ def main():
              "wd": torch.empty((w.E, w.f, w.d), dtype=tdt, device=dev)}
     share_weights(W, world)
     x_np = rank_x(w, rank)
-    x = to_dev(x_np)
+    x = to_dev(x_np, dev)
     bias = configs.make_bias(w)
-    bias_d = None if bias is None else to_dev(bias)
-    cfg = moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype=w.storage)
-    rows = w.T * w.top_k
-    tdt = cfg.torch_dtype
-    buf = {
-        "idx": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
-        "w": torch.empty((w.T, 2), dtype=torch.float32, device=dev),
-        "h": torch.empty((rows, w.f), dtype=tdt, device=dev),
-        "y": torch.empty((rows, w.d), dtype=torch.float32, device=dev),
-        "out": torch.empty((w.T, w.d), dtype=tdt, device=dev),
-        "ws": torch.empty((max(moe.dispatch_workspace_size(cfg), 16),), dtype=torch.uint8, device=dev),
-    }
-    disp = {"counts_raw": torch.empty(8, dtype=torch.int32, device=dev),
-            "counts_kept": torch.empty(8, dtype=torch.int32, device=dev),
-            "offsets": torch.empty(9, dtype=torch.int32, device=dev),
-            "perm": torch.empty(rows, dtype=torch.int32, device=dev),
-            "slot_of": torch.empty((w.T, 2), dtype=torch.int32, device=dev),
-            "row_scale": torch.empty(rows, dtype=torch.float32, device=dev),
-            "x_perm": torch.empty((rows, w.d), dtype=tdt, device=dev)}
+    bias_d = None if bias is None else to_dev(bias, dev)
     stream = torch.cuda.current_stream(dev)
-    names = ["router", "dispatch", "gate_up", "down", "combine"]
-    qw = moe.QuantizedExperts(cfg, W["wg"], W["wu"], W["wd"]) if args.int8 else None
-    ws8 = (torch.empty((max(moe.lib.moe_expert_ffn_w8_workspace_size(cfg.ref), 16),), dtype=torch.uint8, device=dev)
-           if args.int8 else None)
-    # the one-call layer's kernels: bf16 tensor-core batches sum the down outputs into token
-    # order (zero + down + rounding pass, no y buffer, no separate combine)
-    fused = (qw is None and not args.unfused and w.storage == "bf16" and w.T * 2 > 64 * w.E and w.d % 256 == 0)
-    if fused:
-        buf["dc_ws"] = torch.empty(moe.lib.moe_expert_down_combine_workspace_size(cfg.ref), dtype=torch.uint8,
-                                   device=dev)
-    # router 1, dispatch 3 + gather 1, gate/up 1, down 1, combine 1 (int8 experts: + 2 row-code passes
-    # and the partial sum);
-    # fused: router 1, dispatch 3 + gather 1, gate/up 1, zero + down + rounding 3 (9)
-    launches_per_step = 11 if args.int8 else (9 if fused else 8)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        moe.router_topk(cfg, x, W["wr"], bias_d, topk_idx=buf["idx"], topk_w=buf["w"])
-        if ev:
-            ev[1].record(stream)
-        moe.dispatch(cfg, x, buf["idx"], buf["w"], out=disp, ws=buf["ws"])
-        if ev:
-            ev[2].record(stream)
-        if fused:
-            moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
-            if ev:
-                ev[3].record(stream)
-            moe.expert_down_combine(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], disp["perm"],
-                                    out=buf["out"], ws=buf["dc_ws"])
-            if ev:
-                ev[4].record(stream)
-                ev[5].record(stream)
-            return
-        if qw is not None:
-            # int8 experts: gate/up and down in one call (both timed under "gate_up")
-            moe.expert_ffn_w8(cfg, disp["x_perm"], disp["offsets"], qw, disp["row_scale"], y=buf["y"], ws=ws8)
-        else:
-            moe.expert_gate_up(cfg, disp["x_perm"], disp["offsets"], W["wg"], W["wu"], h=buf["h"])
-        if ev:
-            ev[3].record(stream)
-        if qw is None:
-            moe.expert_down(cfg, buf["h"], disp["offsets"], W["wd"], disp["row_scale"], y=buf["y"])
-        if ev:
-            ev[4].record(stream)
-        moe.combine(cfg, buf["y"], disp["slot_of"], buf["w"], weights_applied=True, out=buf["out"])
-        if ev:
-            ev[5].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    n_kept = int(disp["offsets"][-1].item())
-    counts_kept = disp["counts_kept"].cpu().tolist()
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    uuid = ""
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
-    clocks = ClockSampler(uuid)
-    clocks.start()
-    time.sleep(0.5)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    # a pipeline wait that ran out of time sets the device error word: such a run is invalid
-    device_error = moe.get_device_error()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    ms_total = t_start.elapsed_time(t_end)
-    per_kernel = {n: 0.0 for n in names}
-    for e in evs:
-        for j, n in enumerate(names):
-            per_kernel[n] += e[j].elapsed_time(e[j + 1])
-    per_kernel = {n: v / args.steps for n, v in per_kernel.items()}
-    ms_total = max_over_ranks(ms_total, dev, world)
-    ms_step = ms_total / args.steps
-    tokens = world * w.T * args.steps
-    value = throughput(world, w.T, args.steps, ms_total)
-    flops_step = 2.0 * w.T * w.d * w.E + 6.0 * n_kept * w.d * w.f
-    tflops = world * flops_step * args.steps / (ms_total / 1000.0) / 1e12
-
+    run = LayerRun(moe, w, W, x, bias_d, dev, stream, int8=args.int8, unfused=args.unfused)
+    cfg, tdt = run.cfg, run.cfg.torch_dtype
+    res = run.time(args.steps, args.warmup, world)
     peaks, peak_src = load_peaks()
+    summ = layer_summary(w, res, peaks, peak_src, world, args.steps)
+    n_kept, per_kernel = res["n_kept"], res["per_kernel"]
     gu_flops = 4.0 * n_kept * w.d * w.f
-    gu_ms = per_kernel["gate_up"]
-    achieved = gu_flops / (gu_ms / 1000.0) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    gu_name = "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)"
-    roofline = {"bound": "tensor", "kernel": gu_name,
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
-                "traffic": measured_traffic(w.name),
+    roofline = {"bound": "tensor", "kernel": "grouped_gemm_tc_kernel<gate_up> (SwiGLU epilogue)",
+                "achieved": summ["gate_up"]["tflops"], "peak": summ["peak_tflops"], "unit": "TFLOP/s",
+                "frac": summ["gate_up"]["frac"], "peak_source": summ["peak_rule"],
+                "traffic": measured_traffic(w.name, "gate_up"),
                 "traffic_unit": "bytes per launch (dram read + write, ncu)",
                 "algorithmic": f"4*d*f*N_kept = {gu_flops:.4e} FLOP per launch (N_kept={n_kept})",
-                "down": {"achieved": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12,
-                         "frac": 2.0 * n_kept * w.d * w.f / (per_kernel['down'] / 1000.0) / 1e12 / peak}}
-
-    line = {"metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "down": dict(summ["down"], kernel="grouped_gemm_tc_kernel<down> (routing-weight scatter epilogue)",
+                             traffic=measured_traffic(w.name, "down"))}
+    line = {"metric": "MoE-layer tokens/s", "value": summ["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.storage == "bf16" else "f32",
             "data": "synthetic (seeded Philox4x32-10 normal inputs, random-init weights)",
-            "config": dict(workload_config(w), expert_weights="int8" if args.int8 else w.storage), "tflops": tflops,
-            "tensor_frac_layer": tflops / peak,
-            "kernels_ms": per_kernel,
-            "hbm_steps": hbm_steps(w, n_kept, per_kernel, fused, peaks),
-            "gemm_tiles": args.tiles, "device_error": device_error,
+            "config": dict(workload_config(w), expert_weights="int8" if args.int8 else w.storage),
+            "tflops": summ["tflops"], "tensor_frac_layer": summ["tensor_frac_layer"],
+            "kernels_ms": per_kernel, "hbm_steps": hbm_steps(w, n_kept, per_kernel, run.fused, peaks),
+            "gemm_tiles": args.tiles, "device_error": res["device_error"],
             "path": ("down-combine fused: down sums into token order (its time includes the zeroing and "
-                     "rounding passes; combine 0)") if fused else "separate down and combine",
-            "counts_kept": counts_kept, "n_kept": n_kept, "dropped": 2 * w.T - n_kept,
-            "imbalance_max_over_mean_kept": max(counts_kept) / (sum(counts_kept) / len(counts_kept)),
-            "expert_utilization": [c * w.E / max(sum(counts_kept), 1) for c in counts_kept],
-            "gpu_launches": launches_per_step * args.steps, "roofline": roofline, "clocks": clk}
+                     "rounding passes; combine 0)") if run.fused else "separate down and combine",
+            "counts_kept": res["counts_kept"], "n_kept": n_kept, "dropped": summ["dropped"],
+            "imbalance_max_over_mean_kept": summ["imbalance_max_over_mean_kept"],
+            "expert_utilization": [c * w.E / max(sum(res["counts_kept"]), 1) for c in res["counts_kept"]],
+            "gpu_launches": run.launches_per_step * args.steps, "roofline": roofline, "clocks": res["clocks"]}
+    del run
 
-    # ---- end to end: host x in, host out, through the C entry points with host buffers.
-    # Headline: moe_layer_forward_host_batches, one batch per step, every step's x copied
-    # in and its out copied back inside the timed region (overlapped with the compute of
-    # the neighbouring steps).  Also reported: the one-batch call, which waits per batch.
     if not args.no_e2e:
-        ws_full = torch.empty(moe.workspace_size_host_batches(cfg), dtype=torch.uint8, device=dev)
-        x_host = torch.from_numpy(np.ascontiguousarray(x_np))
-        x_host = (x_host.view(torch.bfloat16) if w.storage == "bf16" else x_host).pin_memory()
-        out_ring = [torch.empty((w.T, w.d), dtype=tdt).pin_memory() for _ in range(2)]
-
-        def run_batches(n):
-            moe.layer_forward_host_batches(cfg, [x_host] * n, W["wr"], W["wg"], W["wu"], W["wd"],
-                                           [out_ring[i % 2] for i in range(n)], ws_full, logit_bias=bias_d,
-                                           stream=stream)
-
-        run_batches(args.warmup)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        run_batches(args.steps)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(a.elapsed_time(b), dev, world)
-        nbytes = w.T * w.d * (2 if w.storage == "bf16" else 4)
-        # the one-batch entry point (copy in, layer, copy out, wait) for comparison
-        single_steps = min(args.steps, 10)
-        moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
-                               logit_bias=bias_d, stream=stream)
-        if world > 1:
-            dist.barrier()
-        a.record(stream)
-        for _ in range(single_steps):
-            moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
-                                   logit_bias=bias_d, stream=stream)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        single_ms = max_over_ranks(a.elapsed_time(b), dev, world) / single_steps
-        line["e2e"] = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
-                       "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms / args.steps,
-                       "api": "moe_layer_forward_host_batches (pinned host x/out, one batch per step, copies "
-                              "overlapped with the neighbouring steps' compute; device-resident weights)",
-                       "one_batch_call": {"ms_per_step": single_ms,
-                                          "value": tokens / args.steps / (single_ms / 1000.0),
-                                          "api": "moe_layer_forward_host (copy in, layer, copy out, wait)"}}
-        del ws_full
-
-    # ---- decode (weight streaming) on the same Grok-shape weights
+        line["e2e"] = e2e_bench(moe, w, cfg, W, x_np, bias_d, dev, stream, args, world)
     if not args.no_decode and w.name == "grok_prefill" and not args.shape:
         line["decode"] = decode_bench(moe, W, dev, stream, peaks, peak_src, world)
-
-    # ---- training step (forward that keeps its state + backward) on the same batch
     if (not args.no_train and w.name.startswith("grok_prefill") and w.storage == "bf16" and w.d % 256 == 0
             and w.f % 256 == 0):
-        line["train"] = train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, args.train_steps)
-
+        line["train"] = train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, peak_src, world,
+                                    args.train_steps)
+    if world == 1 and not args.no_configs and w.name == "grok_prefill" and not args.shape and not args.int8:
+        line["per_config"] = per_config(moe, W, dev, stream, peaks, peak_src, summ, line.get("decode"))
     if rank == 0 and world == 1 and not args.no_cpu and host is not None:
-        t, n = oracle_sample(w, host, x_np, args.cpu_tokens, 7)
-        line["cpu_baseline"] = {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"oracle (fp64 numpy): router, top-2 and dispatch over all T={w.T} "
-                                          f"tokens, expert FFN and combine for {n} seeded tokens; "
-                                          f"value = {n} tokens / {t:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline(w, host, x_np, args.cpu_tokens)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
 
-def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, steps):
+def to_dev(a, dev):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+
+def _sampler(dev):
+    import torch
+
+    uuid = ""
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    s = ClockSampler(uuid)
+    s.start()
+    time.sleep(0.3)
+    return s
+
+
+def e2e_bench(moe, w, cfg, W, x_np, bias_d, dev, stream, args, world):
+    """End to end: host x in, host out, through the C entry points with host buffers.
+    Headline: moe_layer_forward_host_batches, one batch per step, every step's x copied
+    in and its out copied back inside the timed region (overlapped with the compute of
+    the neighbouring steps).  Also reported: the one-batch call, which waits per batch."""
+    import torch
+    import torch.distributed as dist
+
+    tdt = cfg.torch_dtype
+    ws_full = torch.empty(moe.workspace_size_host_batches(cfg), dtype=torch.uint8, device=dev)
+    x_host = torch.from_numpy(np.ascontiguousarray(x_np))
+    x_host = (x_host.view(torch.bfloat16) if w.storage == "bf16" else x_host).pin_memory()
+    out_ring = [torch.empty((w.T, w.d), dtype=tdt).pin_memory() for _ in range(2)]
+
+    def run_batches(n):
+        moe.layer_forward_host_batches(cfg, [x_host] * n, W["wr"], W["wg"], W["wu"], W["wd"],
+                                       [out_ring[i % 2] for i in range(n)], ws_full, logit_bias=bias_d,
+                                       stream=stream)
+
+    run_batches(args.warmup)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    run_batches(args.steps)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), dev, world)
+    nbytes = w.T * w.d * (2 if w.storage == "bf16" else 4)
+    tokens = world * w.T * args.steps
+    # the one-batch entry point (copy in, layer, copy out, wait) for comparison
+    single_steps = min(args.steps, 10)
+    moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
+                           logit_bias=bias_d, stream=stream)
+    if world > 1:
+        dist.barrier()
+    a.record(stream)
+    for _ in range(single_steps):
+        moe.layer_forward_host(cfg, x_host, W["wr"], W["wg"], W["wu"], W["wd"], out_ring[0], ws_full,
+                               logit_bias=bias_d, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    single_ms = max_over_ranks(a.elapsed_time(b), dev, world) / single_steps
+    del ws_full
+    return {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms / args.steps,
+            "api": "moe_layer_forward_host_batches (pinned host x/out, one batch per step, copies "
+                   "overlapped with the neighbouring steps' compute; device-resident weights)",
+            "one_batch_call": {"ms_per_step": single_ms, "value": tokens / args.steps / (single_ms / 1000.0),
+                               "api": "moe_layer_forward_host (copy in, layer, copy out, wait)"}}
+
+
+def per_config(moe, W_grok, dev, stream, peaks, peak_src, grok_summary, decode):
+    """Every configuration of the workload list, each timed with its own clock
+    record: the mid bf16 layer and the tiny fp32 layer on their own weights, the
+    skewed Grok layer on the (identical) Grok weights already resident, the Grok
+    prefill headline and the Grok decode calls as measured above."""
+    out = {"grok_prefill": {k: grok_summary[k] for k in ("tokens_per_s", "ms_per_step", "tflops", "gate_up",
+                                                          "down", "n_kept", "dropped", "expert0_share_raw",
+                                                          "imbalance_max_over_mean_kept", "peak_rule")}}
+    out["grok_prefill"]["note"] = "the headline workload (value, roofline and clocks of this line)"
+    plan = (("mid_bf16", None, 1000, 20), ("grok_skew", W_grok, 10, 3), ("tiny_f32", None, 1000, 20))
+    for name, W, steps, warm in plan:
+        w = configs.WORKLOADS[name]
+        if W is None:
+            W = {"wr": to_dev(configs.make_router(w), dev), "wg": to_dev(configs.make_w_gate(w), dev),
+                 "wu": to_dev(configs.make_w_up(w), dev), "wd": to_dev(configs.make_w_down(w), dev)}
+        bias = configs.make_bias(w)
+        run = LayerRun(moe, w, W, to_dev(configs.make_x(w), dev), None if bias is None else to_dev(bias, dev), dev,
+                       stream)
+        s = layer_summary(w, run.time(steps, warm), peaks, peak_src, 1, steps)
+        s["gpu_launches"] = run.launches_per_step * steps
+        if name == "tiny_f32":
+            s["note"] = ("parity case: fp32 experts on the CUDA cores (exact FFMA, no tensor cores), so the "
+                         "bf16 tensor fractions do not apply")
+            for k in ("tensor_frac_layer", "gate_up", "down", "peak_tflops", "peak_rule"):
+                s.pop(k, None)
+        out[name] = s
+        del run
+    if decode:
+        out["grok_decode"] = {k: decode[k] for k in ("ms_per_call", "tokens_per_s", "achieved_gbs", "frac",
+                                                     "peak_gbs", "bound", "clocks") if k in decode}
+        out["grok_decode"]["int8_weights"] = {k: decode["int8_weights"][k]
+                                              for k in ("ms_per_call", "tokens_per_s", "achieved_gbs", "frac")}
+    return out
+
+
+def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, peak_src, world, steps):
     """Forward-for-training + backward of the layer; backward FLOPs = 12*d*f per kept row
-    (dH, dX over gate and up, and the three weight gradients) + 4*T*d*E for the router."""
+    (dH, dX over gate and up, and the three weight gradients) + 4*T*d*E for the router.
+    Per-kernel times come from the library's phase events (moe_profile_phases)."""
     import torch
 
     from synth import normal
@@ -560,23 +784,44 @@ def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, world, steps
         step()
     torch.cuda.synchronize(dev)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    clocks = _sampler(dev)
+    w0 = time.monotonic()
     for i in range(steps):
         step(evs[i])
     torch.cuda.synchronize(dev)
+    clk = clocks.stop(window=(w0, time.monotonic()))
     fwd = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs) / steps, dev, world)
     bwd = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evs) / steps, dev, world)
+    # per-kernel breakdown on separate steps (the phase events add a few us per kernel)
+    moe.profile_phases(True)
+    moe.profile_read()
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize(dev)
+    ph = moe.profile_read()
+    moe.profile_phases(False)
     bwd_flops = 12.0 * n_kept * d * f + 4.0 * cfg.T * d * E
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak, rule = tensor_peak(peaks, peak_src, clk)
     tf = bwd_flops / (bwd / 1000.0) / 1e12
+    unit_flops = {"fwd_gate_up": 4.0 * n_kept * d * f, "fwd_down": 2.0 * n_kept * d * f,
+                  "bwd_dh": 2.0 * n_kept * d * f, "bwd_dx": 4.0 * n_kept * d * f, "bwd_wg_down": 2.0 * n_kept * d * f,
+                  "bwd_wg_gate": 2.0 * n_kept * d * f, "bwd_wg_up": 2.0 * n_kept * d * f}
+    kernels = {}
+    for name, (ms, calls) in ph.items():
+        if calls:
+            k = {"ms": ms / calls}
+            if name in unit_flops:
+                k["tflops"] = unit_flops[name] / (k["ms"] / 1000.0) / 1e12
+                k["frac"] = k["tflops"] / peak
+            kernels[name] = k
     res = {"steps": steps, "forward_train_ms": fwd, "backward_ms": bwd,
            "tokens_per_s": world * cfg.T / ((fwd + bwd) / 1000.0),
-           "backward_tflops": tf, "backward_frac": tf / peak,
+           "backward_tflops": tf, "backward_frac": tf / peak, "peak_tflops": peak, "peak_rule": rule,
            "backward_algorithmic": "12*d*f*N_kept + 4*T*d*E FLOP", "gpu_launches_per_step": 8 + 10,
-           "grad_dtype": "fp32 weight gradients, bf16 dx"}
+           "kernels": kernels, "kernels_note": "per-kernel times from phase events on separate steps",
+           "grad_dtype": "fp32 weight gradients, bf16 dx", "clocks": clk}
     del ws, grads
     return res
-
-
 def graph_decode(moe, cfg, W, xs, out, ws, dev, stream, calls, eager_ms):
     import torch
 
@@ -626,11 +871,14 @@ def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
     torch.cuda.synchronize(dev)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    clocks = _sampler(dev)
+    w0 = time.monotonic()
     a.record(stream)
     for i in range(w.calls):
         moe.layer_forward(cfg, xs[i], W["wr"], W["wg"], W["wu"], W["wd"], out=out, stats=stats, ws=ws)
     b.record(stream)
     torch.cuda.synchronize(dev)
+    clk = clocks.stop(window=(w0, time.monotonic()))
     ms = a.elapsed_time(b)
     # experts used per call (counted after timing, on a second pass)
     n_used = 0
@@ -644,7 +892,7 @@ def decode_bench(moe, W, dev, stream, peaks, peak_src, world):
     res = {"workload": w.name, "calls": w.calls, "ms_per_call": ms / w.calls,
            "tokens_per_s": w.T * w.calls / (ms / 1000.0), "expert_weight_gb_per_call": weight_bytes / w.calls / 1e9,
            "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
-           "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm",
+           "peak_source": f"{peak_src} hbm_gbs", "bound": "hbm", "clocks": clk,
            "kernel": "decode_gemm_kernel (weights on the MMA M side)"}
     # the same calls replayed from a CUDA graph: the layer's launches are captured once
     # and each call copies its x into the captured input buffer, then replays

@@ -1,7 +1,9 @@
 """Host-side parts of bench.py, on CPU: the reference arm (which runs the oracle
 on the host) prints one JSON line of the contract's shape, stops at its
-wall-clock budget and runs on rank 0 only; the DRAM-traffic lookup reports the
-committed capture only while the kernel sources hash to the captured version."""
+wall-clock budget and runs on rank 0 only; the oracle's layer time is
+extrapolated per kept assignment; the tensor peak follows the run's clock; the
+DRAM-traffic lookup reports the committed capture only while the kernel
+sources hash to the captured version."""
 from __future__ import annotations
 
 import hashlib
@@ -32,12 +34,44 @@ def test_reference_arm_prints_one_contract_line():
     assert j["impl"] == "reference" and j["metric"] == "MoE-layer tokens/s" and j["unit"] == "tokens/s"
     assert j["value"] > 0 and j["higher_is_better"] is True and j["n_gpus"] == 1
     assert j["steps"] == 3 and j["steps_requested"] == 3 and j["warmup"] == 1
-    # value = tokens timed / time timed, with --ref-tokens (2) tokens per step
-    assert abs(j["value"] - 2 * 1000.0 / j["ms_per_step"]) <= 1e-9 * j["value"]
+    # value = the layer's T tokens over the oracle's (extrapolated) layer time per step
+    assert abs(j["value"] - 64 * 1000.0 / j["ms_per_step"]) <= 1e-9 * j["value"]
     cb = j["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["unit"] == "tokens/s" and cb["cores"] >= 1
+    assert cb["nproc"] >= 1
     assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert j["config"]["workload"] == "tiny_f32" and j["config"]["T"] == 64
+
+
+def test_oracle_layer_time_extrapolates_per_kept_assignment():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import configs
+
+    w = configs.scaled(configs.WORKLOADS["mid_bf16"], name="small", T=96, d=64, f=128)
+    host = dict(wr=configs.make_router(w), wg=configs.make_w_gate(w), wu=configs.make_w_up(w),
+                wd=configs.make_w_down(w))
+    r = bench.oracle_layer_time(w, host, configs.make_x(w), 16, 3, threads=1)
+    assert r["sample_tokens"] == 16 and 0 < r["kept_in_sample"] <= 32 and r["threads"] == 1
+    assert r["extrapolation"] == r["n_kept"] / r["kept_in_sample"]
+    assert abs(r["layer_s"] - (r["route_s"] + r["ffn_sample_s"] * r["extrapolation"])) <= 1e-12
+    assert abs(r["tokens_per_s"] - w.T / r["layer_s"]) <= 1e-9 * r["tokens_per_s"]
+
+
+def test_tensor_peak_follows_the_run_clock():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "clocks_under_load": {"sm_mhz_median": 1400}}
+    p, rule = bench.tensor_peak(peaks, "measured", {"sm_mhz": 1940.0, "sm_max_mhz": 1965.0})
+    assert p == 1600.0 and "burst" in rule
+    p, rule = bench.tensor_peak(peaks, "measured", {"sm_mhz": 1200.0, "sm_max_mhz": 1965.0})
+    assert p == 1400.0 * 1200.0 / 1400.0 and "sustained" in rule
+    # never above the burst figure
+    p, _ = bench.tensor_peak(peaks, "measured", {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0})
+    assert p == 1600.0
+    p, _ = bench.tensor_peak({"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}, "measured", {})
+    assert p == 1400.0
 
 
 def test_reference_arm_stops_at_its_budget():
@@ -65,15 +99,20 @@ def test_traffic_lookup_follows_the_kernel_sources(tmp_path, monkeypatch):
     for src in bench.KERNEL_SOURCES:
         with open(src, "rb") as fh:
             h.update(fh.read())
-    good = tmp_path / "good.md"
-    good.write_text(f"capture\n    kernel_sources_sha256: {h.hexdigest()}\n    gate_up_dram_bytes_per_launch: 123456\n")
-    stale = tmp_path / "stale.md"
-    stale.write_text("capture\n    kernel_sources_sha256: " + "0" * 64 + "\n    gate_up_dram_bytes_per_launch: 123456\n")
+    body = {"workloads": {"grok_prefill": {"gate_up": {"dram_bytes_per_launch": 123456}}}}
+    good = tmp_path / "good.json"
+    good.write_text(json.dumps(dict(body, kernel_sources_sha256=h.hexdigest())))
+    stale = tmp_path / "stale.json"
+    stale.write_text(json.dumps(dict(body, kernel_sources_sha256="0" * 64)))
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(good))
     assert bench.measured_traffic("grok_prefill") == 123456.0
-    assert bench.measured_traffic("mid_bf16") is None  # captured on the Grok prefill workload only
+    assert bench.measured_traffic("grok_prefill", "down") is None
+    assert bench.measured_traffic("mid_bf16") is None  # no capture of that workload
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(stale))
     assert bench.measured_traffic("grok_prefill") is None
+    # every header the grouped GEMM kernel includes is hashed
+    names = {os.path.basename(p) for p in bench.KERNEL_SOURCES}
+    assert {"ffn_tc.cu", "tc_ptx.cuh", "common.cuh", "internal.h"} <= names
 
 
 def test_clock_sampler_parses_and_filters_by_gpu(tmp_path, monkeypatch):
@@ -100,6 +139,6 @@ def test_clock_sampler_parses_and_filters_by_gpu(tmp_path, monkeypatch):
         if len(s.rows) >= 3:
             break
         time.sleep(0.05)
-    r = s.stop()
+    r = s.stop(window=(0.0, time.monotonic()))
     assert r["samples"] == 3 and r["sm_mhz"] == 1250.0 and r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 1001.0
