@@ -15,7 +15,8 @@ unweighted outputs and the source's combine applies the weights.
 
 The phases (ep_prepare, ep_plan, ep_experts, ep_finish) are separate so that a
 caller can run the exchanges with any transport; layer_forward_ep runs them
-with torch.distributed (NCCL on GPUs).
+with torch.distributed: NCCL moves device memory directly, a host backend
+(gloo) moves the rows through host memory.
 """
 from __future__ import annotations
 
@@ -102,17 +103,31 @@ def ep_finish(cfg: Config, y_back, state, stream=None):
     return combine(cfg, y_back, state["disp"]["slot_of"], state["w"], weights_applied=False, stream=stream)
 
 
+def _host_transport(t, group=None):
+    """True when the group's backend moves only host tensors (gloo) and t is on a GPU:
+    the exchange then goes through host memory (NCCL moves device memory itself)."""
+    return t.is_cuda and dist.get_backend(group) != "nccl"
+
+
 def _all_to_all_rows(send, send_splits, recv_splits, group=None):
-    out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype, device=send.device)
-    dist.all_to_all_single(out, send.contiguous(), recv_splits, send_splits, group=group)
-    return out
+    host = _host_transport(send, group)
+    src = send.contiguous().cpu() if host else send.contiguous()
+    out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype, device=src.device)
+    a, b = out, src
+    if src.dtype == torch.bfloat16 and dist.get_backend(group) != "nccl":
+        # a host backend has no 16-bit float type: the rows travel as int32 pairs
+        # of their bits (rows hold an even number of values)
+        a, b = out.view(torch.int32), src.view(torch.int32)
+    dist.all_to_all_single(a, b, recv_splits, send_splits, group=group)
+    return out.to(send.device) if host else out
 
 
 def gather_table(counts, group=None):
     """table[p, e] = counts of rank p, on the host."""
     world = dist.get_world_size(group)
-    parts = [torch.empty_like(counts) for _ in range(world)]
-    dist.all_gather(parts, counts.contiguous(), group=group)
+    c = counts.contiguous().cpu() if _host_transport(counts, group) else counts.contiguous()
+    parts = [torch.empty_like(c) for _ in range(world)]
+    dist.all_gather(parts, c, group=group)
     return torch.stack(parts).cpu().numpy()
 
 

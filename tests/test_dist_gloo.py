@@ -150,6 +150,11 @@ def _ep_worker(rank, world, port, q):
         experts = np.repeat(np.arange(8), disp["counts_kept"])
         rows = torch.from_numpy(np.stack([np.full(n, rank), disp["perm"], experts], 1).astype(np.int64))
         recv = _all_to_all_rows(rows[:sum(plan["send_splits"])], plan["send_splits"], plan["recv_splits"])
+        # the same rows in bf16 (small integers are exact; 4 columns, as bf16 rows travel in int32 pairs)
+        rows16 = torch.cat([rows, torch.zeros((n, 1), dtype=torch.int64)], 1).to(torch.bfloat16)
+        recv16 = _all_to_all_rows(rows16[:sum(plan["send_splits"])], plan["send_splits"], plan["recv_splits"])
+        assert recv16.dtype == torch.bfloat16
+        assert torch.equal(recv16[:, :3].to(torch.int64), recv) and not recv16[:, 3].any()
         grouped = recv.numpy()[plan["fwd"]]
         back = _all_to_all_rows(torch.from_numpy(grouped[plan["inv"]]), plan["recv_splits"], plan["send_splits"])
         q.put((rank, table, grouped, plan["offsets"], back.numpy(), rows.numpy()))

@@ -2,12 +2,19 @@
 layer_forward_ep in lockstep, and the two all-to-alls are done in-process by
 slicing (no collective; the GPU kernels involved never wait on each other).
 Every rank's output is checked against the oracle on that rank's batch, with
-the bf16 bar of the single-GPU layer."""
+the bf16 bar of the single-GPU layer.  Then layer_forward_ep itself runs end
+to end in two processes that share the GPU, exchanging over gloo through host
+memory (only the host-side collectives wait on the other rank): each rank's
+output must equal the virtual ranks' bit for bit."""
 from __future__ import annotations
+
+import os
+import socket
 
 import numpy as np
 import pytest
 import torch
+import torch.multiprocessing as mp
 
 import oracle
 import sparse_moe_layer_07_b200 as moe
@@ -80,3 +87,77 @@ def test_expert_parallel_ranks_match_the_oracle(world, skew):
         rounded = oracle.to_f64(synth.round_bf16(pre).reshape(pre.shape))
         assert np.array_equal(outs[r].float().cpu().numpy().astype(np.float64), rounded)
     assert moe.get_device_error() == 0
+
+
+def _free_port():
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _ep_case(world):
+    return configs.scaled(W["grok_skew"], name=f"ep_e2e{world}", T=300, d=256, f=384, capacity_factor=1.25)
+
+
+def _ep_batch(w, rank):
+    return configs.make_x(w) if rank == 0 else normal(configs.SEED, configs.TID_X + 1000 * rank, (w.T, w.d),
+                                                        dtype="bf16")
+
+
+def _ep_worker(rank, world, port, q):
+    import sys
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from sparse_moe_layer_07_b200.expert_parallel import layer_forward_ep
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=120))
+    try:
+        torch.cuda.set_device(0)
+        w = _ep_case(world)
+        L = LayerInputs(w, x=_ep_batch(w, rank))
+        D = L.dev
+        out = layer_forward_ep(L.cfg, D["x"], D["wr"], D["wg"], D["wu"], D["wd"], logit_bias=D["bias"])
+        torch.cuda.synchronize()
+        q.put((rank, out.view(torch.int16).cpu().numpy(), moe.get_device_error()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_layer_forward_ep_end_to_end_two_processes():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    try:
+        for _ in range(world):
+            r, out, err = q.get(timeout=300)
+            got[r] = (out, err)
+    finally:
+        for p in procs:
+            p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    # the same ranks in lockstep in this process, exchanges by slicing
+    w = _ep_case(world)
+    L0 = LayerInputs(w)
+    D, cfg = L0.dev, L0.cfg
+    states = [ep_prepare(cfg, to_dev(_ep_batch(w, r)), D["wr"], D["bias"]) for r in range(world)]
+    table = np.stack([st["counts"].cpu().numpy() for st in states])
+    plans = [ep_plan(table, r, world) for r in range(world)]
+    x_recv = [torch.cat([states[p]["disp"]["x_perm"][_splits_start(plans[p]["send_splits"])[q_]:][
+        :plans[p]["send_splits"][q_]] for p in range(world)]) for q_ in range(world)]
+    y_recv = [ep_experts(cfg, x_recv[q_], plans[q_], D["wg"], D["wu"], D["wd"]) for q_ in range(world)]
+    for r in range(world):
+        back = torch.cat([y_recv[q_][_splits_start(plans[q_]["recv_splits"])[r]:][:plans[q_]["recv_splits"][r]]
+                          for q_ in range(world)])
+        want = ep_finish(cfg, back, states[r]).view(torch.int16).cpu().numpy()
+        out, err = got[r]
+        assert err == 0
+        assert np.array_equal(out, want), r
