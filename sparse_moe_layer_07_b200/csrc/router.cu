@@ -132,10 +132,13 @@ __global__ void __launch_bounds__(kWarps * 32) router_top2_split_kernel(const Ti
 // quarter q).  Every wait is bounded; a timeout flags the device error word.
 constexpr int kRtM = 64;
 constexpr int kRtBK = 64;
-constexpr int kRtStages = 11;  // with the receive buffer: two CTAs fit one SM's shared memory
+constexpr int kRtKB = 2;       // K blocks per stage: one TMA box of [2 blocks][64 rows][64]
+constexpr int kRtStages = 5;   // with the receive buffer: two CTAs fit one SM's shared memory
 constexpr int kRtParts = 4;             // K quarters
-constexpr int kRtA = kRtM * kRtBK * 2;  // 8 KB of x per stage
-constexpr int kRtB = kE * kRtBK * 2;    // 1 KB of W_r per stage (one 8-row swizzle atom)
+constexpr int kRtA1 = kRtM * kRtBK * 2;  // 8 KB of x per K block
+constexpr int kRtB1 = kE * kRtBK * 2;    // 1 KB of W_r per K block (one 8-row swizzle atom)
+constexpr int kRtA = kRtKB * kRtA1;
+constexpr int kRtB = kRtKB * kRtB1;
 constexpr int kRtRecv = kRtParts * kRtM * kE * 4;  // quarter sums received by the first CTA
 constexpr int kRtSmem = 1024 + kRtStages * (kRtA + kRtB) + kRtRecv + 256;
 constexpr uint32_t kRtIdesc = ptx::idesc_bf16_f32(kRtM, kE, false, false);
@@ -197,8 +200,12 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
     // ---------------------------------------------------------------- producer
     const uint64_t once = policy_evict_first();
     const uint64_t keep = policy_evict_last();
+    // stage i holds K blocks kb0 + kRtKB i .. + kRtKB - 1 (a box may run past this
+    // CTA's range or the tensor's end: those blocks are loaded, or zero-filled,
+    // and not multiplied)
+    const int n_st = (n_kb + kRtKB - 1) / kRtKB;
     int i = 0;
-    for (; i < n_kb; ++i) {
+    for (; i < n_st; ++i) {
       const int s = i % kRtStages;
       const uint32_t ph = (uint32_t)(i / kRtStages) & 1u;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
@@ -207,8 +214,8 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
         break;
       }
       mbar_arrive_expect_tx(&full[s], kRtA + kRtB);
-      tma_load_2d_hint(sA + s * kRtA, &tmx, &full[s], (kb0 + i) * kRtBK, m0, once);
-      tma_load_2d_hint(sB + s * kRtB, &tmw, &full[s], (kb0 + i) * kRtBK, 0, keep);
+      tma_load_3d_hint(sA + s * kRtA, &tmx, &full[s], 0, m0, kb0 + kRtKB * i, once);
+      tma_load_3d_hint(sB + s * kRtB, &tmw, &full[s], 0, 0, kb0 + kRtKB * i, keep);
     }
     // drain: every issued load must land before the CTA can exit
     const int first = i > kRtStages ? i - kRtStages : 0;
@@ -218,9 +225,8 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
     // ---------------------------------------------------------------- MMA issuer
     bool issued = false;
     int j = j0;
-    for (int i = 0; i < n_kb; ++i) {
-      const int kb = kb0 + i;
-      while (kb >= rt_part_begin(j + 1, num_kb)) ++j;  // the quarter this K block belongs to
+    const int n_st = (n_kb + kRtKB - 1) / kRtKB;
+    for (int i = 0; i < n_st; ++i) {
       const int s = i % kRtStages;
       const uint32_t ph = (uint32_t)(i / kRtStages) & 1u;
       if (!mbar_wait(&full[s], ph, abort_flag)) {
@@ -229,14 +235,20 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      const uint32_t a_addr = smem_u32(sA + s * kRtA);
-      const uint32_t b_addr = smem_u32(sB + s * kRtB);
-      const uint32_t d_tmem = tmem_base + (uint32_t)(kE * (j - j0));
-      const bool first_of_part = kb == rt_part_begin(j, num_kb);
 #pragma unroll
-      for (int kk = 0; kk < kRtBK / 16; ++kk)
-        umma_bf16(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024), sw128_desc(b_addr + kk * 32, 16, 1024),
-                  kRtIdesc, (first_of_part && kk == 0) ? 0u : 1u);
+      for (int u = 0; u < kRtKB; ++u) {
+        const int kb = kb0 + kRtKB * i + u;
+        if (kb >= kb1) break;
+        while (kb >= rt_part_begin(j + 1, num_kb)) ++j;  // the quarter this K block belongs to
+        const uint32_t a_addr = smem_u32(sA + s * kRtA + u * kRtA1);
+        const uint32_t b_addr = smem_u32(sB + s * kRtB + u * kRtB1);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(kE * (j - j0));
+        const bool first_of_part = kb == rt_part_begin(j, num_kb);
+#pragma unroll
+        for (int kk = 0; kk < kRtBK / 16; ++kk)
+          umma_bf16(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024), sw128_desc(b_addr + kk * 32, 16, 1024),
+                    kRtIdesc, (first_of_part && kk == 0) ? 0u : 1u);
+      }
       issued = true;
       umma_commit(&empty[s]);
     }
@@ -305,14 +317,16 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
 
 cudaError_t launch_router_tc(const moe_config_t& c, const void* x, const void* wr, const float* bias, float* logits,
                              int32_t* idx, float* w, cudaStream_t s, const Ctx& ctx) {
+  // 3-D views {64 columns, rows, K block}: a box of kRtKB blocks lands as kRtKB
+  // consecutive [rows][64] tiles, each a run of 128-byte swizzle atoms
   CUtensorMap tx, tw;
-  const uint64_t x_dims[2] = {(uint64_t)c.d, (uint64_t)c.T};
-  const uint64_t w_dims[2] = {(uint64_t)c.d, (uint64_t)kE};
-  const uint64_t str[1] = {(uint64_t)c.d * 2};
-  const uint32_t x_box[2] = {kRtBK, kRtM};
-  const uint32_t w_box[2] = {kRtBK, kE};
-  if (!encode_tmap(&tx, x, 2, x_dims, str, x_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&tw, wr, 2, w_dims, str, w_box, CU_TENSOR_MAP_SWIZZLE_128B))
+  const uint64_t x_dims[3] = {(uint64_t)kRtBK, (uint64_t)c.T, (uint64_t)(c.d / kRtBK)};
+  const uint64_t w_dims[3] = {(uint64_t)kRtBK, (uint64_t)kE, (uint64_t)(c.d / kRtBK)};
+  const uint64_t str[2] = {(uint64_t)c.d * 2, (uint64_t)kRtBK * 2};
+  const uint32_t x_box[3] = {kRtBK, kRtM, kRtKB};
+  const uint32_t w_box[3] = {kRtBK, kE, kRtKB};
+  if (!encode_tmap(&tx, x, 3, x_dims, str, x_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tw, wr, 3, w_dims, str, w_box, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtSmem);
   if (e != cudaSuccess) return e;

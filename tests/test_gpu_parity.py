@@ -30,6 +30,8 @@ SMALL = {
     "bf16_no_drop": (W["mid_bf16"], dict(T=513, d=512, f=640, capacity_factor=4.0)),
     "bf16_skew_drop": (W["grok_skew"], dict(T=1024, d=256, f=512)),
     "bf16_pair_ragged": (W["mid_bf16"], dict(T=1500, d=512, f=768)),
+    # enough down tiles for the 256-column down pass (smaller batches take 128-column tiles)
+    "bf16_down_wide": (W["mid_bf16"], dict(T=4608, d=1024, f=256, capacity_factor=4.0)),
     # at most 64 rows per expert on average: the weight-streaming (swap-AB) kernel
     "bf16_stream_no_drop": (W["mid_bf16"], dict(T=96, d=256, f=384, capacity_factor=4.0)),
     "bf16_stream_ragged": (W["mid_bf16"], dict(T=250, d=384, f=512)),
