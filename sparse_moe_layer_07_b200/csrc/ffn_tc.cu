@@ -758,17 +758,6 @@ cudaError_t launch_tc_gate_up(const moe_config_t& c, const void* x_perm, const i
   return launch_grouped<kGateUp, 256>(ta, tg, tu, args, s, ctx);
 }
 
-// Output columns per down tile: 256, or 128 when 256-column tiles would fill
-// fewer than two waves of the persistent grid (a mostly empty last wave costs
-// up to half the kernel there; 128-column tiles double the tile count).  The
-// estimate uses the config only (T * top_k rows at most, one partial block per
-// expert), so the choice does not depend on the routing.
-int down_tile_cols(const moe_config_t& c, const Ctx& ctx) {
-  if (c.d % 256 != 0) return 128;
-  const int64_t row_blocks = (slot_rows(c) + BM - 1) / BM + c.E;
-  return row_blocks * (c.d / 256) < 2 * (int64_t)ctx.num_sms ? 128 : 256;
-}
-
 cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
                            const float* row_scale, float* y, cudaStream_t s, const Ctx& ctx) {
   const int64_t rows = slot_rows(c);
@@ -795,12 +784,9 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
   args.save_g = nullptr;
   args.save_u = nullptr;
   args.err = ctx.err;
-  if (c.d % 256 == 0 && use_pair_tiles(c)) {
+  if (c.d % 256 == 0) {
     args.n_tiles = (int)(c.d / 256);
-    return launch_pair<kDown, false>(ta, tw, tw, args, s, ctx);
-  }
-  if (down_tile_cols(c, ctx) == 256) {
-    args.n_tiles = (int)(c.d / 256);
+    if (use_pair_tiles(c)) return launch_pair<kDown, false>(ta, tw, tw, args, s, ctx);
     return launch_grouped<kDown, 256>(ta, tw, tw, args, s, ctx);
   }
   args.n_tiles = (int)(c.d / 128);
@@ -835,16 +821,9 @@ cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const i
   args.save_g = nullptr;
   args.save_u = nullptr;
   args.err = ctx.err;
-  if (use_pair_tiles(c)) {
-    args.n_tiles = (int)(c.d / 256);
-    return launch_pair<kDown, true>(ta, tw, tw, args, s, ctx);
-  }
-  if (down_tile_cols(c, ctx) == 256) {
-    args.n_tiles = (int)(c.d / 256);
-    return launch_grouped<kDown, 256, true>(ta, tw, tw, args, s, ctx);
-  }
-  args.n_tiles = (int)(c.d / 128);
-  return launch_grouped<kDown, 128, true>(ta, tw, tw, args, s, ctx);
+  args.n_tiles = (int)(c.d / 256);
+  if (use_pair_tiles(c)) return launch_pair<kDown, true>(ta, tw, tw, args, s, ctx);
+  return launch_grouped<kDown, 256, true>(ta, tw, tw, args, s, ctx);
 }
 
 }  // namespace moe
