@@ -170,9 +170,11 @@ __device__ __forceinline__ void epilogue_rows(const TcArgs& args, int n_rows, in
         p[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                            silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
       if (valid) {
+        // streaming stores: H is read back by the next launch, not by this one, so
+        // its lines should not push the operand tiles out of L2 (1-2% faster)
         uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) __stcs(d4 + i, make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]));
         if (args.save_g) {
           // training: keep the pre-activations for the backward pass
           const int64_t o = (int64_t)(row0 + r) * args.ld_out + n0 + c * 32;
