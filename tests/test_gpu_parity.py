@@ -291,3 +291,20 @@ def test_router_does_not_depend_on_the_batch():
         assert torch.equal(l2, lg[t0:t0 + n]), (t0, n)
         assert torch.equal(i2, idx[t0:t0 + n]) and torch.equal(w2, wts[t0:t0 + n]), (t0, n)
     assert moe.get_device_error() == 0
+
+
+@pytest.mark.parametrize("d", [128, 384, 640, 896])
+def test_router_uneven_quarters(d):
+    """Hidden sizes of 2, 6, 10 and 14 K blocks of 64: quarters that are empty
+    or of unequal length, CTAs with an odd number of blocks (their last
+    two-block box runs into the next CTA's range), one, two or four CTAs per
+    tile (1 to 20000 tokens); against the oracle's fp32 bound and top-2."""
+    for T in (1, 63, 65, 3000, 8192, 20000):
+        w = configs.scaled(W["grok_skew"], name=f"router_d{d}_T{T}", T=T, d=d, f=128)
+        L = LayerInputs(w)
+        idx, wts, lg = moe.router_topk(L.cfg, L.dev["x"], L.dev["wr"], L.dev["bias"], want_logits=True)
+        torch.cuda.synchronize()
+        g = {"idx": idx.cpu().numpy(), "w": wts.cpu().numpy(), "logits": lg.cpu().numpy().astype(np.float64)}
+        tie, mismatch = check_routing(L, g, oracle.router_logits(L.x, L.wr, L.bias))
+        assert mismatch.sum() <= tie.sum()
+    assert moe.get_device_error() == 0
