@@ -64,6 +64,27 @@ def _check(L, g, tokens, name):
     return ref
 
 
+def _bench_launches_equal(L, g):
+    """The launch configuration the benchmark times (router, dispatch, gate/up, and
+    the down pass summing into token order with one rounding pass), and the
+    one-call layer, give the bits of the step-by-step path checked above."""
+    import sparse_moe_layer_07_b200 as moe
+
+    c, D = L.cfg, L.dev
+    idx, wts, _ = moe.router_topk(c, D["x"], D["wr"], D["bias"])
+    disp = moe.dispatch(c, D["x"], idx, wts)
+    h = moe.expert_gate_up(c, disp["x_perm"], disp["offsets"], D["wg"], D["wu"])
+    out = moe.expert_down_combine(c, h, disp["offsets"], D["wd"], disp["row_scale"], disp["perm"])
+    del h
+    torch.cuda.synchronize()
+    assert torch.equal(out, g["out"])
+    del out
+    one = moe.layer_forward(c, D["x"], D["wr"], D["wg"], D["wu"], D["wd"], logit_bias=D["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(one, g["out"])
+    assert moe.get_device_error() == 0
+
+
 def test_grok_prefill_full_size(grok):
     host, dev = grok
     w = W["grok_prefill"]
@@ -72,6 +93,7 @@ def test_grok_prefill_full_size(grok):
     np.testing.assert_array_equal(g["counts_kept"], g["counts_raw"])  # cf = E/k: nothing dropped
     assert int(g["offsets"][-1]) == 2 * w.T
     _check(L, g, _sample(w.T, 62, 11), "grok_prefill")
+    _bench_launches_equal(L, g)
 
 
 def test_grok_skew_full_size(grok):
@@ -84,6 +106,7 @@ def test_grok_skew_full_size(grok):
     partly = np.nonzero((g["slot_of"] < 0).any(1))[0]
     extra = np.random.default_rng(5).choice(partly, size=min(16, partly.size), replace=False)
     _check(L, g, _sample(w.T, 46, 12, extra), "grok_skew")
+    _bench_launches_equal(L, g)
 
 
 def test_grok_decode_full_size(grok):
