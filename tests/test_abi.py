@@ -249,3 +249,30 @@ def test_binding_checks_element_counts_and_types(moe):
         moe.layer_forward(c, x.to(torch.bfloat16), wr, w[:4], w, w)
     with pytest.raises(ValueError, match="logit_bias must be"):
         moe.router_topk(c, x.to(torch.bfloat16), wr, logit_bias=torch.zeros(8, dtype=torch.float64))
+
+
+def test_utilization_arguments_checked_before_launch(moe):
+    p = ctypes.c_void_p(16)  # never dereferenced: the call must fail on E first
+    for E in (0, -1, 65):
+        assert moe.lib.moe_expert_utilization(p, E, p, p, None) == 1  # MOE_ERR_INVALID_ARG
+    assert moe.lib.moe_expert_utilization(None, 8, p, p, None) == 1
+    assert moe.lib.moe_expert_utilization(p, 8, None, p, None) == 1
+    assert moe.lib.moe_expert_utilization(p, 8, p, None, None) == 1
+
+
+def test_phase_profile_read_without_events(moe):
+    """With nothing recorded, a read fills zeros for the phases asked for, takes
+    NULL arrays and shorter arrays, and rejects a negative count."""
+    assert moe.PHASES[7] == "bwd_dh" and len(moe.PHASES) == 14
+    moe.profile_phases(True)
+    try:
+        got = moe.profile_read()
+        assert set(got) == set(moe.PHASES) and all(v == (0.0, 0) for v in got.values())
+        ms = (ctypes.c_float * 3)(9.0, 9.0, 9.0)
+        calls = (ctypes.c_int32 * 3)(7, 7, 7)
+        assert moe.lib.moe_profile_read(ms, calls, 3) == 0
+        assert list(ms) == [0.0, 0.0, 0.0] and list(calls) == [0, 0, 0]
+        assert moe.lib.moe_profile_read(None, None, 14) == 0
+        assert moe.lib.moe_profile_read(ms, calls, -1) == 1
+    finally:
+        moe.profile_phases(False)
