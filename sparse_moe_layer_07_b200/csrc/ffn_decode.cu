@@ -94,8 +94,6 @@ __device__ __forceinline__ DTile decode_dtile(const DSched& s, int L, int n_cb) 
   return t;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
-
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
@@ -279,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j)
             if (j0 + j < t.rows)
               H[(int64_t)(t.m0 + j0 + j) * args.ld_out + n] =
-                  __float2bfloat16_rn(silu_mul(__uint_as_float(g[j]), __uint_as_float(u[j])));
+                  __float2bfloat16_rn(silu_mul_fast(__uint_as_float(g[j]), __uint_as_float(u[j])));
         }
       } else {
         float* Y = static_cast<float*>(args.out);

@@ -137,8 +137,6 @@ __device__ __forceinline__ Tile8 tile8(const Sched8& s, int L, int n_cb, int ksp
   return t;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
-
 __device__ __forceinline__ float code_value(uint32_t hi, uint32_t lo) {
   return fmaf(256.0f, (float)(int)hi, (float)(int)lo);
 }
@@ -344,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float sr = __ldg(args.row_code_scale + row);
               const float g = sg * sr * code_value(gh[j], gl[j]);
               const float u = su * sr * code_value(uh[j], ul[j]);
-              out[row * args.ld_out + n] = silu_mul(g, u);
+              out[row * args.ld_out + n] = silu_mul_fast(g, u);
             }
           }
         }

@@ -133,8 +133,6 @@ __device__ __forceinline__ void build_schedule(Sched& sched, const TcArgs& args,
   if (!ok) flag_error(args.err, MOE_DEVERR_OFFSETS);
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
-
 // Source token of grouped row `row` for the fused variants (0 for rows past the
 // kept ones, which are computed and never stored; a bad index is flagged).
 __device__ __forceinline__ int source_token(const TcArgs& args, int row, int n_rows) {
@@ -158,17 +156,30 @@ __device__ __forceinline__ void epilogue_rows(const TcArgs& args, int n_rows, in
   if (MODE == kGateUp) {
     __nv_bfloat16* H = static_cast<__nv_bfloat16*>(args.out);
     __nv_bfloat16* dst_row = H + (int64_t)(row0 + r) * args.ld_out + n0;
-#pragma unroll 1
-    for (int c = 0; c < n_cols / 32; ++c) {
-      uint32_t g[32], u[32];
-      tmem_ld32(tacc + c * 32, g);
-      tmem_ld32(tacc + u_off + c * 32, u);
+    // 32-column chunks (n_cols <= 128); the TMEM loads of chunk c + 1 are in
+    // flight while chunk c is computed and stored (the loop is unrolled so the
+    // two register sets stay in registers)
+    const int nch = n_cols / 32;
+    uint32_t gb[2][32], ub[2][32];
+    tmem_ld32(tacc, gb[0]);
+    tmem_ld32(tacc + u_off, ub[0]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c >= nch) break;
       tmem_wait_ld();
+      tmem_regs_ready(gb[c & 1]);
+      tmem_regs_ready(ub[c & 1]);
+      if (c + 1 < nch) {
+        tmem_ld32(tacc + (c + 1) * 32, gb[(c + 1) & 1]);
+        tmem_ld32(tacc + u_off + (c + 1) * 32, ub[(c + 1) & 1]);
+      }
+      const uint32_t(&g)[32] = gb[c & 1];
+      const uint32_t(&u)[32] = ub[c & 1];
       uint32_t p[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        p[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                           silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+        p[i] = pack_bf16x2(silu_mul_fast(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                           silu_mul_fast(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
       if (valid) {
         // streaming stores: H is read back by the next launch, not by this one, so
         // its lines should not push the operand tiles out of L2 (1-2% faster)
