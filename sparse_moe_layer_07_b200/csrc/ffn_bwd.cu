@@ -271,63 +271,56 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
-    // Lane 0 waits and issues; for the weight gradients all 32 lanes zero the
-    // rows past the expert's end in its last K block first.
-    constexpr bool kMN = MODE == kWG;
-    constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kMN, kMN);
-    constexpr uint32_t IDESC_M64 = idesc_bf16_f32(64, BN, kMN, kMN);
-    uint32_t it = 0, tc = 0;
-    bool ok = true, issued = false;
-    for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
-      const Tile t = decode_tile<MODE>(sched, args, L);
-      // a row block of at most 64 rows (an expert's last) runs M = 64 MMAs
-      const uint32_t idesc = (MODE != kWG && t.rows <= 64) ? IDESC_M64 : IDESC;
-      const uint32_t buf = tc & 1u;
-      const uint32_t tph = (tc >> 1) & 1u;
-      int got = 1;
-      if (lane == 0) got = mbar_wait(&tempty[buf], tph ^ 1u, abort_flag) ? 1 : 0;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + buf * kAccStride;
-      for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1u;
-        // weight gradients: every lane observes the landed stage itself, since
-        // lanes may overwrite part of it below
-        if (lane == 0 || MODE == kWG) got = mbar_wait(&full[s], ph, abort_flag) ? 1 : 0;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
+    // Lane 0 alone waits and issues, as in the forward GEMMs: a warp-wide loop
+    // with a shuffle and a warp sync per K block held the dH and dx kernels
+    // 25-35% below the MMA rate.  For the weight gradients it also zeroes the
+    // rows past the expert's end in the expert's last K block.
+    if (lane == 0) {
+      constexpr bool kMN = MODE == kWG;
+      constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kMN, kMN);
+      constexpr uint32_t IDESC_M64 = idesc_bf16_f32(64, BN, kMN, kMN);
+      uint32_t it = 0, tc = 0;
+      bool ok = true, issued = false;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
+        const Tile t = decode_tile<MODE>(sched, args, L);
+        // a row block of at most 64 rows (an expert's last) runs M = 64 MMAs
+        const uint32_t idesc = (MODE != kWG && t.rows <= 64) ? IDESC_M64 : IDESC;
+        const uint32_t buf = tc & 1u;
+        const uint32_t tph = (tc >> 1) & 1u;
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        // K steps of 16 rows issued for this block: the expert's last block issues
-        // only the steps that hold its rows, and the rows of the last such step
-        // past the expert's end (next expert's rows, or past the kept rows) are
-        // zeroed in both operands first (each row is 128 bytes of every chunk).
-        int ksteps = BK / 16;
-        if (MODE == kWG) {
-          const int valid = t.nrows - kb * BK;
-          if (valid < BK) {
-            ksteps = (valid + 15) / 16;
-            const int pad = ksteps * 16 - valid;
-            if (pad > 0) {
-              const int per_chunk = pad * 8;  // 16-byte pieces
-              for (int i = lane; i < 6 * per_chunk; i += 32) {
-                const int c = i / per_chunk;
-                const int j = i - c * per_chunk;
-                uint8_t* chunk = c < 2 ? sA + s * A_BYTES + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
-                *reinterpret_cast<uint4*>(chunk + valid * 128 + j * 16) = make_uint4(0u, 0u, 0u, 0u);
-              }
-              fence_proxy_async_smem();
-            }
-            __syncwarp();
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * kAccStride;
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
           }
-        }
-        if (lane == 0) {
+          // K steps of 16 rows issued for this block: the expert's last block
+          // issues only the steps that hold its rows, and the rows of the last
+          // such step past the expert's end (next expert's rows, or past the kept
+          // rows) are zeroed in both operands first (a row is 128 bytes of every
+          // 8 KB chunk, so the swizzle does not matter).
+          int ksteps = BK / 16;
+          if (MODE == kWG) {
+            const int valid = t.nrows - kb * BK;
+            if (valid < BK) {
+              ksteps = (valid + 15) / 16;
+              const int pad = ksteps * 16 - valid;
+              if (pad > 0) {
+                for (int c = 0; c < 6; ++c) {
+                  uint8_t* chunk = c < 2 ? sA + s * A_BYTES + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
+                  uint4* z = reinterpret_cast<uint4*>(chunk + valid * 128);
+                  for (int j = 0; j < pad * 8; ++j) z[j] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+              }
+            }
+          }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
@@ -347,12 +340,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
           issued = true;
           umma_commit(&empty[s]);
         }
-        __syncwarp();
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(&tfull[buf]);
-    }
-    if (lane == 0) {
       if (!ok) {
         flag_error(args.err, MOE_DEVERR_TIMEOUT);
         *abort_flag = 1;
