@@ -255,10 +255,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
               tma_load_3d_hint(b + c * CHUNK, first ? &tmB0 : &tmB1, &full[s], k0, t.n0 + 64 * c, t.e, keep);
           } else {
             const int r0 = t.row0 + kb * BK;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) tma_load_2d_hint(a + c * CHUNK, &tmA0, &full[s], t.m0 + 64 * c, r0, keep);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tma_load_2d_hint(b + c * CHUNK, &tmB0, &full[s], t.n0 + 64 * c, r0, keep);
+            tma_load_3d_hint(a, &tmA0, &full[s], 0, r0, t.m0 / 64, keep);
+            tma_load_3d_hint(b, &tmB0, &full[s], 0, r0, t.n0 / 64, keep);
           }
         }
       }
@@ -594,7 +592,18 @@ cudaError_t launch_bwd_wgrad(const moe_config_t& c, const void* a_rows, int64_t 
   const int64_t rows = slot_rows(c);
   if (rows == 0 || M % BM != 0 || N % BN != 0) return rows == 0 ? cudaSuccess : cudaErrorInvalidValue;
   CUtensorMap ta, tb, to;
-  if (!map_rows(&ta, a_rows, rows, M, 64) || !map_rows(&tb, b_rows, rows, N, 64)) return cudaErrorInvalidValue;
+  {
+    // [rows, C] viewed as [C / 64 chunks][rows][64]: one box = nch chunks of 64 x 64
+    const uint64_t a_dims[3] = {64, (uint64_t)rows, (uint64_t)(M / 64)};
+    const uint64_t a_str[2] = {(uint64_t)M * 2, 128};
+    const uint32_t a_box[3] = {64, 64, 2};
+    const uint64_t b_dims[3] = {64, (uint64_t)rows, (uint64_t)(N / 64)};
+    const uint64_t b_str[2] = {(uint64_t)N * 2, 128};
+    const uint32_t b_box[3] = {64, 64, 4};
+    if (!encode_tmap(&ta, a_rows, 3, a_dims, a_str, a_box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap(&tb, b_rows, 3, b_dims, b_str, b_box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   // dW [E * M, N] fp32, stored 32 x 32 at a time from the swizzled staging tiles
   const uint64_t o_dims[2] = {(uint64_t)N, (uint64_t)c.E * M};
   const uint64_t o_str[1] = {(uint64_t)N * 4};
