@@ -546,7 +546,7 @@ def main():
     ap.add_argument("--shape", default=None, help="T,d,f override of the workload (profiling cases)")
     ap.add_argument("--int8", action="store_true", help="int8 expert weights (weight-only, per-channel scales)")
     ap.add_argument("--no-train", action="store_true", help="skip the training pair (forward + backward)")
-    ap.add_argument("--train-steps", type=int, default=5)
+    ap.add_argument("--train-steps", type=int, default=20)
     ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair"],
                     help="tile shape of the bf16 grouped GEMMs")
     ap.add_argument("--unfused", action="store_true",
@@ -724,7 +724,7 @@ def per_config(moe, W_grok, dev, stream, peaks, peak_src, grok_summary, decode):
                                                           "down", "n_kept", "dropped", "expert0_share_raw",
                                                           "imbalance_max_over_mean_kept", "peak_rule")}}
     out["grok_prefill"]["note"] = "the headline workload (value, roofline and clocks of this line)"
-    plan = (("mid_bf16", None, 1000, 20), ("grok_skew", W_grok, 10, 3), ("tiny_f32", None, 1000, 20))
+    plan = (("mid_bf16", None, 3000, 20), ("grok_skew", W_grok, 30, 3), ("tiny_f32", None, 2000, 20))
     for name, W, steps, warm in plan:
         w = configs.WORKLOADS[name]
         if W is None:
