@@ -452,7 +452,10 @@ class LayerRun:
 
     def time(self, steps, warmup, world=1):
         """W untimed steps, then K steps between a barrier + synchronize on both
-        sides, clocks sampled during the timed region; the max over ranks."""
+        sides, clocks sampled during the timed region; the max over ranks.
+        Per-kernel times come from up to 100 further steps with CUDA events
+        between the calls (kept out of the timed steps, where they would
+        serialise the launches)."""
         import torch
         import torch.distributed as dist
 
@@ -463,7 +466,6 @@ class LayerRun:
         n_kept = int(self.disp["offsets"][-1].item())
         counts_kept = self.disp["counts_kept"].cpu().tolist()
         counts_raw = self.disp["counts_raw"].cpu().tolist()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
         uuid = ""
         try:
             uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -478,9 +480,12 @@ class LayerRun:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         w0 = time.monotonic()
+        # no events between the calls inside the timed steps: an event between two
+        # launches would stop the next kernel's launch from overlapping the
+        # previous kernel's exit (programmatic dependent launch)
         t_start.record(stream)
         for i in range(steps):
-            self.step(evs[i])
+            self.step()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
         w1 = time.monotonic()
@@ -490,11 +495,17 @@ class LayerRun:
             dist.barrier()
         clk = clocks.stop(window=(w0, w1))
         ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev, world)
+        # per-kernel times on separate steps, with events between the calls
+        n_k = min(steps, 100)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_k)]
+        for i in range(n_k):
+            self.step(evs[i])
+        torch.cuda.synchronize(dev)
         per_kernel = {n: 0.0 for n in self.NAMES}
         for e in evs:
             for j, n in enumerate(self.NAMES):
                 per_kernel[n] += e[j].elapsed_time(e[j + 1])
-        per_kernel = {n: v / steps for n, v in per_kernel.items()}
+        per_kernel = {n: v / n_k for n, v in per_kernel.items()}
         return {"ms_total": ms_total, "ms_step": ms_total / steps, "per_kernel": per_kernel, "n_kept": n_kept,
                 "counts_kept": counts_kept, "counts_raw": counts_raw, "device_error": device_error, "clocks": clk}
 

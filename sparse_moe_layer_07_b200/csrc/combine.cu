@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 __global__ void __launch_bounds__(256) zero_kernel(float4* __restrict__ p, int64_t n4) {
+  pdl_wait();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x)
     p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256) zero_kernel(float4* __restrict__ p, int64
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) round_out_kernel(const float4* __restrict__ src, void* __restrict__ out,
                                                         int64_t n4) {
+  pdl_wait();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     const float4 a = __ldg(src + i);
     if (kBf16Out) {
@@ -106,18 +108,18 @@ unsigned grid_for(int64_t n4, const Ctx& ctx) {
 cudaError_t launch_zero_rows(const moe_config_t& c, float* out32, cudaStream_t s, const Ctx& ctx) {
   const int64_t n4 = c.T * c.d / 4;
   if (n4 == 0) return cudaSuccess;
-  zero_kernel<<<grid_for(n4, ctx), 256, 0, s>>>(reinterpret_cast<float4*>(out32), n4);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(zero_kernel, dim3(grid_for(n4, ctx)), dim3(256), 0, s, no_extra_attr(),
+                                   reinterpret_cast<float4*>(out32), n4);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_round_out(const moe_config_t& c, const float* out32, void* out, cudaStream_t s, const Ctx& ctx) {
   const int64_t n4 = c.T * c.d / 4;
   if (n4 == 0) return cudaSuccess;
-  if (c.dtype == MOE_BF16)
-    round_out_kernel<true><<<grid_for(n4, ctx), 256, 0, s>>>(reinterpret_cast<const float4*>(out32), out, n4);
-  else
-    round_out_kernel<false><<<grid_for(n4, ctx), 256, 0, s>>>(reinterpret_cast<const float4*>(out32), out, n4);
-  return cudaGetLastError();
+  const cudaError_t e =
+      launch_pdl(c.dtype == MOE_BF16 ? round_out_kernel<true> : round_out_kernel<false>, dim3(grid_for(n4, ctx)),
+                 dim3(256), 0, s, no_extra_attr(), reinterpret_cast<const float4*>(out32), out, n4);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const float* y, const int32_t* slot_of,

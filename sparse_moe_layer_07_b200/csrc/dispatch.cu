@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kBT) dispatch_hist_kernel(const int32_t* __res
   __shared__ int s_cnt[kWarps][kE];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * kBT + threadIdx.x;
+  pdl_wait();
   int e0, e1;
   load_pair(idx, t, T, e0, e1, err);
 #pragma unroll
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
                                                            int32_t* __restrict__ offsets, int32_t* __restrict__ stats) {
   __shared__ int s_total[kE];
   const int lane = threadIdx.x & 31, e = threadIdx.x >> 5;
+  pdl_wait();
   int running = 0;
   for (int64_t b0 = 0; b0 < nblk; b0 += 32) {
     const int64_t b = b0 + lane;
@@ -137,6 +139,7 @@ __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __res
   __shared__ int64_t s_prior[kE];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * kBT + threadIdx.x;
+  pdl_wait();
   int e0, e1;
   load_pair(idx, t, T, e0, e1, err);
   if (threadIdx.x < kE) {
@@ -182,6 +185,7 @@ __global__ void __launch_bounds__(kBT) dispatch_rank_kernel(const int32_t* __res
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
                                                          const int32_t* __restrict__ offsets, int64_t T,
                                                          int64_t row_vec, uint4* __restrict__ x_perm, int* err) {
+  pdl_wait();
   int64_t n = offsets[kE];
   const int lane = threadIdx.x & 31;
   if (n < 0 || n > 2 * T) {
@@ -218,14 +222,20 @@ cudaError_t launch_dispatch(const moe_config_t& c, int64_t cap, const int32_t* i
                             int32_t* stats, cudaStream_t s, const Ctx& ctx, const int32_t* shard_counts,
                             int shard) {
   const int64_t nblk = dispatch_blocks(c);
+  cudaError_t e = cudaSuccess;
   if (nblk > 0) {
-    dispatch_hist_kernel<<<(unsigned)nblk, kBT, 0, s>>>(idx, c.T, block_hist, ctx.err);
+    e = launch_pdl(dispatch_hist_kernel, dim3((unsigned)nblk), dim3(kBT), 0, s, no_extra_attr(), idx, c.T, block_hist,
+                   ctx.err);
+    if (e != cudaSuccess) return e;
   }
-  dispatch_scan_kernel<<<1, 256, 0, s>>>(block_hist, nblk, cap, shard_counts, shard, counts_raw, counts_kept,
-                                          offsets, stats);
+  e = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(256), 0, s, no_extra_attr(), block_hist, nblk, cap,
+                 shard_counts, shard, counts_raw, counts_kept, offsets, stats);
+  if (e != cudaSuccess) return e;
   if (nblk > 0) {
-    dispatch_rank_kernel<<<(unsigned)nblk, kBT, 0, s>>>(idx, w, c.T, cap, shard_counts, shard, block_hist, offsets,
-                                                        perm, slot_of, row_scale, ctx.err);
+    e = launch_pdl(dispatch_rank_kernel, dim3((unsigned)nblk), dim3(kBT), 0, s, no_extra_attr(), idx, w, c.T, cap,
+                   shard_counts, shard, static_cast<const int32_t*>(block_hist), static_cast<const int32_t*>(offsets),
+                   perm, slot_of, row_scale, ctx.err);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -308,9 +318,10 @@ cudaError_t launch_gather(const moe_config_t& c, const void* x, const int32_t* p
   int64_t blocks = (rows + 7) / 8;  // 8 warps per block, one row per warp
   const int64_t cap_blocks = (int64_t)ctx.num_sms * 8;
   if (blocks > cap_blocks) blocks = cap_blocks;
-  gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(x), perm, offsets, c.T, row_vec,
-                                                      static_cast<uint4*>(x_perm), ctx.err);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, no_extra_attr(),
+                                   static_cast<const uint4*>(x), perm, offsets, c.T, row_vec,
+                                   static_cast<uint4*>(x_perm), ctx.err);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 

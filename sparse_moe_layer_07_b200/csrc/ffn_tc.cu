@@ -291,6 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmB0);
     prefetch_tmap(&tmB1);
   }
+  // everything above is local to the CTA; what follows reads the previous kernels' outputs
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -714,8 +716,8 @@ cudaError_t launch_grouped(const CUtensorMap& a, const CUtensorMap& b0, const CU
   auto kern = grouped_gemm_tc_kernel<MODE, MMA_N, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<ctx.num_sms, kThreads, C::SMEM_BYTES, s>>>(a, b0, b1, args);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3(ctx.num_sms), dim3(kThreads), C::SMEM_BYTES, s, no_extra_attr(), a, b0, b1, args);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -7,6 +7,8 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include <utility>
+
 #include "moe.h"
 
 namespace moe {
@@ -49,6 +51,33 @@ struct Ctx {
 
 // Unique id of the current CUDA context (cuCtxGetId); false when none is current.
 bool current_context_id(unsigned long long* id);
+
+// Launch with programmatic stream serialization: the kernel is launched while
+// the previous kernel of the stream is finishing (its launch overlaps that
+// kernel's exit); the kernel calls pdl_wait() before it touches global memory.  `extra` adds one more launch attribute (e.g. a cluster
+// shape) when its id is not cudaLaunchAttributeIgnore.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              const cudaLaunchAttribute& extra, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (extra.id != cudaLaunchAttributeIgnore) attr[n++] = extra;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+inline cudaLaunchAttribute no_extra_attr() {
+  cudaLaunchAttribute a = {};
+  a.id = cudaLaunchAttributeIgnore;
+  return a;
+}
 
 // Rows of the grouped buffers (x_perm, h, y): every assignment may be kept.
 inline int64_t slot_rows(const moe_config_t& c) { return c.T * (int64_t)c.top_k; }

@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
     prefetch_tmap(&tmx);
     prefetch_tmap(&tmw);
   }
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 32);
     tmem_relinquish();
@@ -334,19 +335,12 @@ cudaError_t launch_router_tc(const moe_config_t& c, const void* x, const void* w
   // CTAs per tile: enough that about 1.5 CTAs per SM stream x at once (two fit per SM)
   int nsplit = 1;
   while (nsplit < kRtParts && tiles * nsplit * 2 < (int64_t)ctx.num_sms * 3) nsplit *= 2;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)nsplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(tiles * nsplit), 1, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = kRtSmem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, router_tc_kernel, tx, tw, bias, logits, idx, w, c.T, (int)(c.d / kRtBK), nsplit,
+  cudaLaunchAttribute cluster = {};
+  cluster.id = cudaLaunchAttributeClusterDimension;
+  cluster.val.clusterDim.x = (unsigned)nsplit;
+  cluster.val.clusterDim.y = 1;
+  cluster.val.clusterDim.z = 1;
+  e = launch_pdl(router_tc_kernel, dim3((unsigned)(tiles * nsplit), 1, 1), dim3(128, 1, 1), kRtSmem, s, cluster, tx, tw, bias, logits, idx, w, c.T, (int)(c.d / kRtBK), nsplit,
                          ctx.err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
