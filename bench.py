@@ -450,6 +450,27 @@ class LayerRun:
         moe.combine(cfg, buf["y"], disp["slot_of"], buf["w"], weights_applied=True, out=buf["out"])
         mark(5)
 
+    def router_alone(self, reps=30):
+        """The router kernel timed on its own, each launch after a plain read of a
+        256 MB buffer has replaced L2's contents with clean lines (in the step the
+        router starts with the previous step's output dirty in L2, whose
+        write-back shares the HBM bandwidth).  Median ms over `reps` launches."""
+        import torch
+
+        scratch = torch.ones(256 << 20, dtype=torch.uint8, device=self.dev)
+        times = []
+        for _ in range(reps + 3):
+            scratch.max()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            self.moe.router_topk(self.cfg, self.x, self.W["wr"], self.bias_d, topk_idx=self.buf["idx"],
+                                 topk_w=self.buf["w"])
+            e1.record(self.stream)
+            times.append((e0, e1))
+        torch.cuda.synchronize(self.dev)
+        del scratch
+        return float(sorted(a.elapsed_time(b) for a, b in times[3:])[reps // 2])
+
     def time(self, steps, warmup, world=1):
         """W untimed steps, then K steps between a barrier + synchronize on both
         sides, clocks sampled during the timed region; the max over ranks.
@@ -631,6 +652,14 @@ def main():
             "imbalance_max_over_mean_kept": summ["imbalance_max_over_mean_kept"],
             "expert_utilization": [c * w.E / max(sum(res["counts_kept"]), 1) for c in res["counts_kept"]],
             "gpu_launches": run.launches_per_step * args.steps, "roofline": roofline, "clocks": res["clocks"]}
+    rt = line["hbm_steps"].get("router")
+    if rt:
+        ms_alone = run.router_alone()
+        gbs = rt["bytes"] / (ms_alone / 1000.0) / 1e9
+        rt["alone"] = {"ms": ms_alone, "gbs": gbs, "frac_hbm": gbs / peaks.get("hbm_gbs", 6650.0),
+                       "note": "the same kernel launched on its own after a 256 MB read has left only clean lines "
+                               "in L2 (median of 30); in the step it starts with the previous step's output "
+                               "dirty in L2"}
     del run
 
     if not args.no_e2e:
