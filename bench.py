@@ -541,6 +541,19 @@ def gemm_roofline(w, res, peaks, src):
     return peak, rule, gu, dn
 
 
+def per_clock(tflops, clocks):
+    """The kernel's rate per SM clock against the nominal dense bf16 rate of a
+    B200 SM (one 128 x 256 x 16 MMA per 128 clocks = 8192 FLOP per clock), at
+    the run's median SM clock.  That median covers the whole step, short kernels
+    included, so it is an upper bound on the GEMM's clock and the fraction a
+    lower bound."""
+    mhz = (clocks or {}).get("sm_mhz")
+    if not mhz or not tflops:
+        return None
+    fpc = tflops * 1e12 / (148 * mhz * 1e6)
+    return {"flop_per_clock_per_sm": fpc, "frac_of_nominal": fpc / 8192.0, "sm_mhz": mhz}
+
+
 def layer_summary(w, res, peaks, src, world, steps):
     """tokens/s, TFLOP/s, GEMM roofline fractions, drops and balance of one timed workload."""
     n = res["n_kept"]
@@ -635,6 +648,7 @@ def main():
                 "frac": summ["gate_up"]["frac"], "peak_source": summ["peak_rule"],
                 "traffic": measured_traffic(w.name, "gate_up"),
                 "traffic_unit": "bytes per launch (dram read + write, ncu)",
+                "per_clock": per_clock(summ["gate_up"]["tflops"], res["clocks"]),
                 "algorithmic": f"4*d*f*N_kept = {gu_flops:.4e} FLOP per launch (N_kept={n_kept})",
                 "down": dict(summ["down"], kernel="grouped_gemm_tc_kernel<down> (routing-weight scatter epilogue)",
                              traffic=measured_traffic(w.name, "down"))}
