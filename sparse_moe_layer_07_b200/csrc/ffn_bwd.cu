@@ -43,7 +43,10 @@ constexpr int BK = 64;
 template <int MODE>
 struct Warps {
   static constexpr int kEpi = 4;
-  static constexpr int kThreads = 64 + 32 * kEpi;
+  // weight gradients: one more warp zeroes the rows past an expert's end in its
+  // last K block, so the MMA warp does not stall on it
+  static constexpr int kZeroWarp = MODE == 2 ? 2 + kEpi : -1;
+  static constexpr int kThreads = 64 + 32 * kEpi + (MODE == 2 ? 32 : 0);
 };
 constexpr int kTmemCols = 512;
 constexpr int kAccStride = 256;
@@ -58,6 +61,9 @@ constexpr int OUT_STAGE = 32 * 32 * 4;
 constexpr int OUT_BYTES = 4 * 2 * OUT_STAGE;
 constexpr int SMEM_BYTES = 1024 + kStages * STAGE + OUT_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// full, empty, zeroed (kStages each), tfull, tempty (2 each), drain, then the
+// TMEM slot, the abort flag and the producer's stage count
+static_assert((3 * kStages + 5) * 8 + 12 <= 256, "barrier area");
 
 enum Mode { kDH = 0, kDX = 1, kWG = 2 };
 
@@ -185,17 +191,24 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* zeroed = drain + 1;  // kWG: stage s of a ragged last K block is zeroed and ready
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(zeroed + S);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // kWG: K blocks whose loads the producer has issued (the zeroing warp waits on
+  // a stage's full barrier only once its loads are issued, so the barrier is at
+  // that K block's phase and not at an earlier phase of the same parity)
+  volatile uint32_t* issued_kb = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
   __shared__ Sched sched;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    *issued_kb = 0;
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&zeroed[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -257,6 +270,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const int r0 = t.row0 + kb * BK;
             tma_load_3d_hint(a, &tmA0, &full[s], 0, r0, t.m0 / 64, keep);
             tma_load_3d_hint(b, &tmB0, &full[s], 0, r0, t.n0 / 64, keep);
+            *issued_kb = it + 1;
           }
         }
       }
@@ -271,13 +285,12 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     // -------------------------------------------------------------- MMA issuer
     // Lane 0 alone waits and issues, as in the forward GEMMs: a warp-wide loop
     // with a shuffle and a warp sync per K block held the dH and dx kernels
-    // 25-35% below the MMA rate.  For the weight gradients it also zeroes the
-    // rows past the expert's end in the expert's last K block.
+    // 25-35% below the MMA rate.
     if (lane == 0) {
       constexpr bool kMN = MODE == kWG;
       constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kMN, kMN);
       constexpr uint32_t IDESC_M64 = idesc_bf16_f32(64, BN, kMN, kMN);
-      uint32_t it = 0, tc = 0;
+      uint32_t it = 0, tc = 0, zphase = 0;  // zphase: parity bit per stage of `zeroed`
       bool ok = true, issued = false;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tc) {
         const Tile t = decode_tile<MODE>(sched, args, L);
@@ -294,30 +307,28 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
-            ok = false;
-            break;
-          }
           // K steps of 16 rows issued for this block: the expert's last block
-          // issues only the steps that hold its rows, and the rows of the last
-          // such step past the expert's end (next expert's rows, or past the kept
-          // rows) are zeroed in both operands first (a row is 128 bytes of every
-          // 8 KB chunk, so the swizzle does not matter).
+          // issues only the steps that hold its rows; when the last such step
+          // also holds rows past the expert's end, the zeroing warp clears them
+          // in both operands and releases the stage on zeroed[s] instead.
           int ksteps = BK / 16;
+          bool ragged = false;
           if (MODE == kWG) {
             const int valid = t.nrows - kb * BK;
             if (valid < BK) {
               ksteps = (valid + 15) / 16;
-              const int pad = ksteps * 16 - valid;
-              if (pad > 0) {
-                for (int c = 0; c < 6; ++c) {
-                  uint8_t* chunk = c < 2 ? sA + s * A_BYTES + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
-                  uint4* z = reinterpret_cast<uint4*>(chunk + valid * 128);
-                  for (int j = 0; j < pad * 8; ++j) z[j] = make_uint4(0u, 0u, 0u, 0u);
-                }
-                fence_proxy_async_smem();
-              }
+              ragged = ksteps * 16 > valid;
             }
+          }
+          if (ragged) {
+            if (!mbar_wait(&zeroed[s], (zphase >> s) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            zphase ^= 1u << s;
+          } else if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
@@ -349,6 +360,52 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         umma_commit(drain);
         mbar_wait(drain, 0, nullptr, 100000000ull);
       }
+    }
+  } else if (warp == Warps<MODE>::kZeroWarp) {
+    // ------------------------------------------------ ragged-row zeroing (kWG)
+    // The tile's last K block may hold rows past the expert's end (the next
+    // expert's rows, or rows past the kept ones): once the stage has landed,
+    // zero those rows of the last 16-row step in all six 8 KB chunks (a row is
+    // 128 bytes of a chunk, so the swizzle does not matter), make the writes
+    // visible to the tensor core and release the stage to the MMA warp.  Every
+    // lane waits for the stage itself, so its stores follow the TMA's.
+    uint32_t it = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      const Tile t = decode_tile<MODE>(sched, args, L);
+      const uint32_t it_last = it + (uint32_t)t.nkb - 1u;
+      it += (uint32_t)t.nkb;
+      if (t.nkb == 0) continue;
+      const int valid = t.nrows - (t.nkb - 1) * BK;
+      const int pad = (valid + 15) / 16 * 16 - valid;
+      if (valid >= BK || pad == 0) continue;
+      const int s = it_last % S;
+      // bounded: the producer issues this K block's loads unless the kernel aborts
+      const uint64_t t0 = globaltimer_ns();
+      bool go = true;
+      while ((int)(*issued_kb - it_last) <= 0) {
+        if (*abort_flag || globaltimer_ns() - t0 > 2000000000ull) {
+          go = false;
+          break;
+        }
+        __nanosleep(32);
+      }
+      if (!go || !mbar_wait(&full[s], (it_last / S) & 1u, abort_flag)) {
+        if (!*abort_flag) {
+          if (lane == 0) flag_error(args.err, MOE_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const int per_chunk = pad * 8;  // 16-byte pieces
+      for (int i = lane; i < 6 * per_chunk; i += 32) {
+        const int c = i / per_chunk;
+        const int j = i - c * per_chunk;
+        uint8_t* chunk = c < 2 ? sA + s * A_BYTES + c * CHUNK : sB + s * B_BYTES + (c - 2) * CHUNK;
+        *reinterpret_cast<uint4*>(chunk + valid * 128 + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&zeroed[s]);
     }
   } else {
     // -------------------------------------------------------------- epilogue
