@@ -3,7 +3,8 @@ on the host) prints one JSON line of the contract's shape, stops at its
 wall-clock budget and runs on rank 0 only; the oracle's layer time is
 extrapolated per kept assignment; the tensor peak follows the run's clock; the
 DRAM-traffic lookup reports the committed capture only while the kernel
-sources hash to the captured version."""
+sources hash to the captured version; the per-clock figure is the rate against
+8192 FLOP per SM clock."""
 from __future__ import annotations
 
 import hashlib
@@ -142,3 +143,19 @@ def test_clock_sampler_parses_and_filters_by_gpu(tmp_path, monkeypatch):
     r = s.stop(window=(0.0, time.monotonic()))
     assert r["samples"] == 3 and r["sm_mhz"] == 1250.0 and r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 1001.0
+
+
+def test_per_clock_rate_against_the_nominal_sm_rate():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    # 148 SMs x 8192 FLOP per clock at 1300 MHz is 1576 TFLOP/s: that rate is 1.0 of nominal
+    full = 148 * 8192 * 1300e6 / 1e12
+    r = bench.per_clock(full, {"sm_mhz": 1300.0})
+    assert abs(r["frac_of_nominal"] - 1.0) < 1e-12 and abs(r["flop_per_clock_per_sm"] - 8192.0) < 1e-9
+    r = bench.per_clock(full / 2, {"sm_mhz": 1300.0})
+    assert abs(r["frac_of_nominal"] - 0.5) < 1e-12
+    # the same rate at a higher clock is a smaller fraction per clock
+    assert bench.per_clock(full, {"sm_mhz": 2600.0})["frac_of_nominal"] == 0.5
+    # no clock record, no figure
+    assert bench.per_clock(full, {"sm_mhz": None}) is None and bench.per_clock(full, None) is None
