@@ -333,9 +333,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + s * B_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (kk >= ksteps) break;
+          auto mma_step = [&](int kk) {
             uint64_t ad, bd;
             if (kMN) {
               ad = sw128_desc(a_addr + kk * 2048, CHUNK, 1024);
@@ -345,6 +343,14 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
               bd = sw128_desc(b_addr + kk * 32, 16, 1024);
             }
             umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          };
+          // full K blocks issue their four steps without a branch: a bound check
+          // inside this loop cost the weight gradients 11% of the MMA rate
+          if (ksteps == BK / 16) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) mma_step(kk);
+          } else {
+            for (int kk = 0; kk < ksteps; ++kk) mma_step(kk);
           }
           issued = true;
           umma_commit(&empty[s]);
