@@ -40,6 +40,13 @@ CASES = {
     # every token routed to experts 0 and 1: experts 2..7 have no rows
     "train_two_experts": (W["mid_bf16"], dict(T=300, d=256, f=256, capacity_factor=4.0,
                                               logit_bias=(60.0, 50.0, 0, 0, 0, 0, 0, 0))),
+    # the same with 256 rows per expert (whole 64-row K blocks of the weight
+    # gradients) and with 272 (a last K block of one whole 16-row step, nothing
+    # to zero)
+    "train_two_experts_k64": (W["mid_bf16"], dict(T=256, d=256, f=256, capacity_factor=4.0,
+                                                  logit_bias=(60.0, 50.0, 0, 0, 0, 0, 0, 0))),
+    "train_two_experts_k16": (W["mid_bf16"], dict(T=272, d=256, f=256, capacity_factor=4.0,
+                                                  logit_bias=(60.0, 50.0, 0, 0, 0, 0, 0, 0))),
 }
 
 
