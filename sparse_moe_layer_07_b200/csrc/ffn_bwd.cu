@@ -18,9 +18,11 @@
 //         dW_down = H^T (w * dout),  dW_gate = X^T dG,  dW_up = X^T dU); K is
 //         the ragged row count: the expert's last K block issues only the
 //         16-row MMA steps that hold its rows, and the rows of the last step
-//         past the expert's end are zeroed in shared memory before the MMA.
-// Pipeline as in ffn_tc.cu: persistent CTAs, warp 0 TMA, warp 1 MMA + TMEM
-// (two 128 x 256 fp32 accumulators), warps 2-5 epilogue; every wait bounded.
+//         past the expert's end are zeroed in shared memory before the MMA
+//         (by warp 6, which only kWG has).
+// Pipeline as in ffn_tc.cu: persistent CTAs, warp 0 TMA, warp 1 MMA (lane 0
+// alone) + TMEM (two 128 x 256 fp32 accumulators), warps 2-5 epilogue; every
+// wait bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
