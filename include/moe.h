@@ -442,6 +442,88 @@ MOE_API moe_status_t moe_expert_utilization(const int32_t* stats, int32_t E, int
 MOE_API moe_status_t moe_profile_phases(int32_t enable);
 MOE_API moe_status_t moe_profile_read(float* ms, int32_t* calls, int32_t n);
 
+/* Expert parallelism over peer memory ("Expert parallelism vs. tensor
+ * parallelism", moe_layer_ep_forward: dispatch to the ranks owning the chosen
+ * experts, expert FFN, combine back on the source rank), with the exchanges
+ * written by the kernels themselves instead of two all-to-alls: the dispatch
+ * kernel stores each kept row straight into the owner's grouped buffer, and
+ * the owner's down projection adds routing_weight * (h @ W_down) straight into
+ * the source rank's fp32 sums.  Rank q owns experts [q*E/W, (q+1)*E/W).
+ *
+ * moe_ep_peers_t lists every rank's exchange buffers as device addresses valid
+ * in the calling process (its own allocations, or other ranks' allocations
+ * mapped with moe_peer_import).  With R = world * T * top_k (every kept row of
+ * every rank may go to one owner) and T the tokens of every rank:
+ *   x_grp[q]  [R, d] cfg->dtype  rows rank q receives, its experts in order,
+ *                                each expert's rows by source rank, then in
+ *                                the source's kept order
+ *   src[q]    [R] int32          source of each of those rows: p * T + t
+ *   scale[q]  [R] fp32           routing weight of each of those rows
+ *   sums[p]   [T, d] fp32        rank p's output sums, by token
+ * One step, on every rank, in this order (the caller puts a barrier across
+ * the ranks at each |, e.g. a one-element NCCL all-reduce on the stream):
+ *   moe_router_topk, moe_dispatch (x_perm NULL), table = every rank's
+ *   counts_kept, moe_ep_dispatch_peers | moe_ep_expert_ffn_peers |
+ *   moe_ep_combine_peers.
+ * The result on rank p equals moe_layer_forward on rank p's tokens bit for bit
+ * in the fused down + combine scope (bf16, d a multiple of 256, top_k 2; every
+ * row's products and its two-term fp32 sum do not depend on which rows share a
+ * tile or on the order of the two adds).  world in {1, 2, 4, 8} (dividing E =
+ * 8) and world * T <= 2^30, else MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG. */
+#define MOE_EP_MAX_WORLD 8
+typedef struct moe_ep_peers_t {
+  int32_t world;
+  int32_t rank;
+  void* x_grp[MOE_EP_MAX_WORLD];
+  int32_t* src[MOE_EP_MAX_WORLD];
+  float* scale[MOE_EP_MAX_WORLD];
+  float* sums[MOE_EP_MAX_WORLD];
+} moe_ep_peers_t;
+
+/* Zeroes sums[rank], then stores each of this rank's kept rows x[perm[r], :]
+ * (with src and scale) into x_grp of the expert's owner, and writes this rank's
+ * grouped offsets as an owner, grp_offsets [E + 1] (experts of other ranks
+ * empty).  table [world, E] int32 (device): row p = counts_kept of rank p;
+ * offsets, perm, row_scale: this rank's moe_dispatch outputs; x [T, d].  A
+ * table row of this rank that disagrees with offsets, or an out-of-range perm
+ * entry, sets MOE_DEVERR_OFFSETS / MOE_DEVERR_SLOT_INDEX and stores nothing for
+ * the rows concerned.  The stores are fenced at system scope before the kernel
+ * ends. */
+MOE_API moe_status_t moe_ep_dispatch_peers(const moe_config_t* cfg, const moe_ep_peers_t* peers,
+                                           const int32_t* table, const void* x, const int32_t* offsets,
+                                           const int32_t* perm, const float* row_scale, int32_t* grp_offsets,
+                                           moe_stream_t stream);
+
+/* This rank's experts over the rows it received: h = silu(x_grp W_gate) *
+ * (x_grp W_up) ([R, f] cfg->dtype, caller's scratch), then for each row
+ * sums[p][t, :] += scale * (h W_down) with p * T + t = src of the row (vector
+ * fp32 atomics into the source's buffer).  grp_offsets from
+ * moe_ep_dispatch_peers; weights [E, d, f] / [E, f, d] (only this rank's
+ * experts are read). */
+MOE_API moe_status_t moe_ep_expert_ffn_peers(const moe_config_t* cfg, const moe_ep_peers_t* peers,
+                                             const int32_t* grp_offsets, const void* w_gate, const void* w_up,
+                                             const void* w_down, void* h, moe_stream_t stream);
+
+/* out [T, d] (cfg->dtype) = sums[rank] rounded once. */
+MOE_API moe_status_t moe_ep_combine_peers(const moe_config_t* cfg, const moe_ep_peers_t* peers, void* out,
+                                          moe_stream_t stream);
+
+/* Peer mappings for moe_ep_peers_t (CUDA IPC).  moe_peer_export describes the
+ * device allocation holding `ptr` (any address inside a cudaMalloc block) so
+ * that another process can map it: moe_peer_import maps it into the calling
+ * process (peer access enabled on first use) and returns the address that
+ * corresponds to `ptr`; moe_peer_release unmaps it (pass the imported address
+ * and its handle).  A handle cannot be imported by the process that exported
+ * it (use the address itself there).  MOE_ERR_CUDA when the runtime refuses
+ * (e.g. memory not from cudaMalloc). */
+typedef struct moe_peer_handle_t {
+  uint8_t ipc[64];
+  uint64_t offset;
+} moe_peer_handle_t;
+MOE_API moe_status_t moe_peer_export(const void* ptr, moe_peer_handle_t* handle);
+MOE_API moe_status_t moe_peer_import(const moe_peer_handle_t* handle, void** ptr);
+MOE_API moe_status_t moe_peer_release(void* ptr, const moe_peer_handle_t* handle);
+
 /* Waits for the current device, returns the device error word (MOE_DEVERR_*
  * bits, 0 when clean) in *code, and clears it when `clear` is non-zero.
  * Returns MOE_ERR_DEVICE_CHECK when the word is non-zero, else MOE_OK. */

@@ -25,6 +25,8 @@ __all__ = [
     "layer_forward_w8", "QuantizedExperts", "w8_workspace_views", "expert_down_combine",
     "layer_forward_host_batches", "workspace_size_host_batches",
     "workspace_size_train", "layer_forward_train", "layer_backward", "route_counts", "dispatch_shard", "gather_rows",
+    "EP_MAX_WORLD", "EpPeers", "ep_dispatch_peers", "ep_expert_ffn_peers", "ep_combine_peers", "peer_export",
+    "peer_import", "peer_release",
     "GEMM_TILES", "set_gemm_tiles", "gemm_tiles", "PHASES", "profile_phases", "profile_read",
 ]
 
@@ -49,6 +51,19 @@ class _CConfig(ctypes.Structure):
                 ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int32),
                 ("reserved", ctypes.c_int32)]
+
+
+EP_MAX_WORLD = 8
+
+
+class _CEpPeers(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("x_grp", ctypes.c_void_p * EP_MAX_WORLD), ("src", ctypes.c_void_p * EP_MAX_WORLD),
+                ("scale", ctypes.c_void_p * EP_MAX_WORLD), ("sums", ctypes.c_void_p * EP_MAX_WORLD)]
+
+
+class _CPeerHandle(ctypes.Structure):
+    _fields_ = [("ipc", ctypes.c_uint8 * 64), ("offset", ctypes.c_uint64)]
 
 
 _BUILD_HINT = "build it with `python sparse_moe_layer_07_b200/build.py`"
@@ -99,6 +114,12 @@ def _load():
         "moe_expert_utilization": ([P, ctypes.c_int32, P, P, P], ctypes.c_int),
         "moe_profile_phases": ([ctypes.c_int32], ctypes.c_int),
         "moe_profile_read": ([P, P, ctypes.c_int32], ctypes.c_int),
+        "moe_ep_dispatch_peers": ([cfgp, ctypes.POINTER(_CEpPeers), P, P, P, P, P, P, P], ctypes.c_int),
+        "moe_ep_expert_ffn_peers": ([cfgp, ctypes.POINTER(_CEpPeers), P, P, P, P, P, P], ctypes.c_int),
+        "moe_ep_combine_peers": ([cfgp, ctypes.POINTER(_CEpPeers), P, P], ctypes.c_int),
+        "moe_peer_export": ([P, ctypes.POINTER(_CPeerHandle)], ctypes.c_int),
+        "moe_peer_import": ([ctypes.POINTER(_CPeerHandle), ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+        "moe_peer_release": ([P, ctypes.POINTER(_CPeerHandle)], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         try:
@@ -366,6 +387,77 @@ def expert_down_combine(cfg: Config, h, offsets, w_down, row_scale, perm, out=No
                                        _dev_ptr(perm), _dev_ptr(out), _dev_ptr(ws), ws.numel(),
                                        _stream(stream, h.device)), "moe_expert_down_combine")
     return out
+
+
+class EpPeers:
+    """``moe_ep_peers_t``: every rank's exchange buffers as addresses valid in
+    this process.  ``addrs[q]`` = (x_grp, src, scale, sums) device addresses of
+    rank q (this process's own tensors, or another rank's mapped with
+    ``peer_import``); ``world`` ranks, this one ``rank``."""
+
+    def __init__(self, world: int, rank: int, addrs):
+        if not 1 <= world <= EP_MAX_WORLD or not 0 <= rank < world or len(addrs) != world:
+            raise ValueError(f"world {world}, rank {rank}, {len(addrs)} address sets")
+        self.world, self.rank = int(world), int(rank)
+        self._c = _CEpPeers()
+        self._c.world, self._c.rank = self.world, self.rank
+        for q, (xg, src, sc, sums) in enumerate(addrs):
+            self._c.x_grp[q], self._c.src[q], self._c.scale[q], self._c.sums[q] = xg, src, sc, sums
+
+    @property
+    def ref(self):
+        return ctypes.byref(self._c)
+
+
+def ep_dispatch_peers(cfg: Config, peers: EpPeers, table, x, disp, grp_offsets=None, stream=None):
+    """Zero this rank's sums and store its kept rows (x[perm]) into the owners'
+    grouped buffers (moe_ep_dispatch_peers).  table [world, E] int32 on the
+    device; disp: this rank's dispatch() result.  Returns grp_offsets [E + 1]."""
+    if grp_offsets is None:
+        grp_offsets = _empty((cfg.E + 1,), torch.int32, table)
+    _expect("table", table, peers.world * cfg.E, torch.int32)
+    _check(lib.moe_ep_dispatch_peers(cfg.ref, peers.ref, _dev_ptr(table), _dev_ptr(x), _dev_ptr(disp["offsets"]),
+                                     _dev_ptr(disp["perm"]), _dev_ptr(disp["row_scale"]), _dev_ptr(grp_offsets),
+                                     _stream(stream, table.device)), "moe_ep_dispatch_peers")
+    return grp_offsets
+
+
+def ep_expert_ffn_peers(cfg: Config, peers: EpPeers, grp_offsets, w_gate, w_up, w_down, h, stream=None):
+    """This rank's experts over the rows it received; the weighted outputs are
+    added into the source ranks' sums (moe_ep_expert_ffn_peers).  h: scratch of
+    world * T * top_k rows of f."""
+    _expect("h", h, peers.world * cfg.T * cfg.top_k * cfg.f, cfg.torch_dtype)
+    _check(lib.moe_ep_expert_ffn_peers(cfg.ref, peers.ref, _dev_ptr(grp_offsets), _dev_ptr(w_gate), _dev_ptr(w_up),
+                                       _dev_ptr(w_down), _dev_ptr(h), _stream(stream, h.device)),
+           "moe_ep_expert_ffn_peers")
+
+
+def ep_combine_peers(cfg: Config, peers: EpPeers, out, stream=None):
+    """out [T, d] = this rank's sums rounded once (moe_ep_combine_peers)."""
+    _expect("out", out, cfg.T * cfg.d, cfg.torch_dtype)
+    _check(lib.moe_ep_combine_peers(cfg.ref, peers.ref, _dev_ptr(out), _stream(stream, out.device)),
+           "moe_ep_combine_peers")
+    return out
+
+
+def peer_export(t) -> bytes:
+    """Handle (72 bytes) that lets another process map the allocation holding t."""
+    h = _CPeerHandle()
+    _check(lib.moe_peer_export(_dev_ptr(t), ctypes.byref(h)), "moe_peer_export")
+    return bytes(h)
+
+
+def peer_import(handle: bytes) -> int:
+    """Maps another process's exported allocation; returns the address matching its tensor."""
+    h = _CPeerHandle.from_buffer_copy(handle)
+    p = ctypes.c_void_p()
+    _check(lib.moe_peer_import(ctypes.byref(h), ctypes.byref(p)), "moe_peer_import")
+    return int(p.value)
+
+
+def peer_release(addr: int, handle: bytes):
+    h = _CPeerHandle.from_buffer_copy(handle)
+    _check(lib.moe_peer_release(ctypes.c_void_p(addr), ctypes.byref(h)), "moe_peer_release")
 
 
 def combine(cfg: Config, y, slot_of, topk_w=None, weights_applied: bool = True, out=None, stream=None):

@@ -79,6 +79,11 @@ struct TcArgs {
   const float* row_scale;  // down only; NULL means 1
   const int32_t* perm;     // fused variants: source token of each row
   int64_t n_tok;           // fused variants: rows of x / out (tokens)
+  // fused down over peer memory: perm holds p * n_tok + t and row t of source
+  // rank p's sums is peer_out[p] + t * ld_out (n_peers == 0: out is the one
+  // destination)
+  int n_peers = 0;
+  float* peer_out[MOE_EP_MAX_WORLD] = {};
   void* save_g;            // gate/up for training: also write G and U (bf16) or NULL
   void* save_u;
   int* err;
@@ -139,7 +144,7 @@ __device__ __forceinline__ void build_schedule(Sched& sched, const TcArgs& args,
 __device__ __forceinline__ int source_token(const TcArgs& args, int row, int n_rows) {
   if (row >= n_rows) return 0;
   const int t = __ldg(args.perm + row);
-  if (t < 0 || (int64_t)t >= args.n_tok) {
+  if (t < 0 || (int64_t)t >= args.n_tok * (args.n_peers > 0 ? args.n_peers : 1)) {
     flag_error(args.err, MOE_DEVERR_SLOT_INDEX);
     return -1;
   }
@@ -208,8 +213,15 @@ __device__ __forceinline__ void epilogue_rows(const TcArgs& args, int n_rows, in
     }
   } else if (kScatter) {
     float* O = static_cast<float*>(args.out);
-    const int tok = valid ? source_token(args, row0 + r, n_rows) : -1;
+    int tok = valid ? source_token(args, row0 + r, n_rows) : -1;
     const bool store = tok >= 0;
+    if (store && args.n_peers > 0) {
+      const int p = tok / (int)args.n_tok;
+      tok -= p * (int)args.n_tok;
+#pragma unroll
+      for (int i = 0; i < MOE_EP_MAX_WORLD; ++i)
+        if (i == p) O = args.peer_out[i];
+    }
     float* dst_row = O + (int64_t)(store ? tok : 0) * args.ld_out + n0;
     const float sc = (store && args.row_scale) ? __ldg(args.row_scale + row0 + r) : 1.0f;
 #pragma unroll 1
@@ -413,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
+    // adds into other GPUs' memory: visible system-wide before the kernel ends
+    if (kScatter && args.n_peers > 0) __threadfence_system();
   }
 
   __syncthreads();
@@ -645,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * buf);
     }
+    if (kScatter && args.n_peers > 0) __threadfence_system();
   }
 
   __syncthreads();
@@ -811,7 +826,7 @@ cudaError_t launch_tc_down(const moe_config_t& c, const void* h, const int32_t* 
 
 cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
                                    const float* row_scale, const int32_t* perm, float* out32, cudaStream_t s,
-                                   const Ctx& ctx) {
+                                   const Ctx& ctx, int n_peers, float* const* peer_out, int64_t peer_tokens) {
   const int64_t rows = slot_rows(c);
   if (rows == 0) return cudaSuccess;
   if (c.d % 256 != 0) return cudaErrorInvalidValue;
@@ -838,6 +853,12 @@ cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const i
   args.save_u = nullptr;
   args.err = ctx.err;
   args.n_tiles = (int)(c.d / 256);
+  if (n_peers > 0) {
+    if (n_peers > MOE_EP_MAX_WORLD || !peer_out || peer_tokens <= 0) return cudaErrorInvalidValue;
+    args.n_peers = n_peers;
+    args.n_tok = peer_tokens;
+    for (int p = 0; p < n_peers; ++p) args.peer_out[p] = peer_out[p];
+  }
   if (use_pair_tiles(c)) return launch_pair<kDown, true>(ta, tw, tw, args, s, ctx);
   return launch_grouped<kDown, 256, true>(ta, tw, tw, args, s, ctx);
 }

@@ -134,10 +134,13 @@ int set_tile_mode(int mode);
 bool use_pair_tiles(const moe_config_t& c);
 
 // Down with the combine fused: adds row_scale * (H W_down) into a zeroed fp32
-// out32 [T, d] by token (perm) instead of writing Y.
+// out32 [T, d] by token (perm) instead of writing Y.  With n_peers > 0 the
+// destinations are other ranks' sums: perm holds p * peer_tokens + t and the
+// row goes to peer_out[p] + t * d (out32 unused).
 cudaError_t launch_tc_down_scatter(const moe_config_t& c, const void* h, const int32_t* offsets, const void* wd,
                                    const float* row_scale, const int32_t* perm, float* out32, cudaStream_t s,
-                                   const Ctx& ctx);
+                                   const Ctx& ctx, int n_peers = 0, float* const* peer_out = nullptr,
+                                   int64_t peer_tokens = 0);
 // Backward of the expert FFNs (bf16, d and f multiples of 256): dG / dU and the
 // routing-weight partials, dx (added into a zeroed fp32 dx32 by token), and
 // the weight gradients dW[e] = A_e^T B_e over each expert's rows ([E, M, N] fp32).

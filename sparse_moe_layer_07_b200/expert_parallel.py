@@ -17,14 +17,25 @@ The phases (ep_prepare, ep_plan, ep_experts, ep_finish) are separate so that a
 caller can run the exchanges with any transport; layer_forward_ep runs them
 with torch.distributed: NCCL moves device memory directly, a host backend
 (gloo) moves the rows through host memory.
+
+layer_forward_ep_peers replaces both all-to-alls with stores into the other
+ranks' memory (moe_ep_dispatch_peers / moe_ep_expert_ffn_peers): the
+dispatch kernel writes each kept row into its owner's grouped buffer, the
+owner's down kernel adds the weighted outputs into the source's fp32 sums, and
+two barriers across the ranks separate the phases.  EpPeerGroup maps the other
+ranks' buffers (CUDA IPC); ep_forward_peers_local runs the same kernels for
+`world` ranks held by one process on one device.
 """
 from __future__ import annotations
+
+import contextlib
 
 import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import Config, combine, dispatch, expert_ffn, gather_rows, router_topk
+from . import (Config, EpPeers, combine, dispatch, ep_combine_peers, ep_dispatch_peers, ep_expert_ffn_peers,
+               expert_ffn, gather_rows, peer_export, peer_import, peer_release, router_topk)
 
 
 def owned_experts(rank: int, world: int, E: int = 8):
@@ -143,3 +154,145 @@ def layer_forward_ep(cfg: Config, x, w_router, w_gate, w_up, w_down, logit_bias=
     y_recv = ep_experts(cfg, x_recv, plan, w_gate, w_up, w_down, stream=stream)
     y_back = _all_to_all_rows(y_recv, plan["recv_splits"], plan["send_splits"], group)
     return ep_finish(cfg, y_back, st, stream=stream)
+
+
+# ---------------------------------------------------------------- peer memory
+
+class EpPeerBuffers:
+    """One rank's exchange buffers for the peer-memory path, carved from one
+    allocation so that a single IPC handle maps them all (the same layout on
+    every rank), plus its local scratch: with R = world * T * top_k rows,
+    x_grp [R, d], src [R] int32, scale [R] fp32, sums [T, d] fp32 (shared), and
+    h [R, f], grp_offsets [E + 1] (local)."""
+
+    def __init__(self, cfg: Config, world: int, device):
+        R = world * cfg.T * cfg.top_k
+        esz = torch.empty((), dtype=cfg.torch_dtype).element_size()
+        sizes = [R * cfg.d * esz, R * 4, R * 4, cfg.T * cfg.d * 4]
+        self.part_offsets, off = [], 0
+        for n in sizes:
+            self.part_offsets.append(off)
+            off += (n + 255) // 256 * 256
+        self.raw = torch.empty((max(off, 256),), dtype=torch.uint8, device=device)
+        o = self.part_offsets
+        self.x_grp = self.raw[o[0]:o[0] + sizes[0]].view(cfg.torch_dtype).view(R, cfg.d)
+        self.src = self.raw[o[1]:o[1] + sizes[1]].view(torch.int32)
+        self.scale = self.raw[o[2]:o[2] + sizes[2]].view(torch.float32)
+        self.sums = self.raw[o[3]:o[3] + sizes[3]].view(torch.float32).view(cfg.T, cfg.d)
+        self.h = torch.empty((R, cfg.f), dtype=cfg.torch_dtype, device=device)
+        self.grp_offsets = torch.empty((cfg.E + 1,), dtype=torch.int32, device=device)
+
+    def addrs(self, base=None):
+        """(x_grp, src, scale, sums) addresses given the allocation's address
+        `base` in this process (default: this rank's own)."""
+        b = self.raw.data_ptr() if base is None else int(base)
+        return tuple(b + o for o in self.part_offsets)
+
+
+def ep_route(cfg: Config, x, w_router, logit_bias=None, stream=None):
+    """Route and dispatch this rank's tokens without gathering x (the peer
+    dispatch reads x itself)."""
+    idx, w, _ = router_topk(cfg, x, w_router, logit_bias, stream=stream)
+    return dispatch(cfg, x, idx, w, gather=False, stream=stream)
+
+
+def ep_forward_peers_local(cfg: Config, xs, w_router, w_gate, w_up, w_down, logit_bias=None, bufs=None,
+                           stream=None):
+    """The peer-memory path for len(xs) ranks held by this process on one
+    device: rank r's tokens xs[r] [T, d], its output returned at [r].  The
+    stream's order stands in for the barriers: every rank's dispatch, then
+    every rank's experts, then every rank's rounding."""
+    world = len(xs)
+    dev = xs[0].device
+    if bufs is None:
+        bufs = [EpPeerBuffers(cfg, world, dev) for _ in range(world)]
+    addrs = [b.addrs() for b in bufs]
+    peers = [EpPeers(world, r, addrs) for r in range(world)]
+    disps = [ep_route(cfg, x, w_router, logit_bias, stream=stream) for x in xs]
+    table = torch.stack([d["counts_kept"] for d in disps])
+    for r in range(world):
+        ep_dispatch_peers(cfg, peers[r], table, xs[r], disps[r], bufs[r].grp_offsets, stream=stream)
+    for r in range(world):
+        ep_expert_ffn_peers(cfg, peers[r], bufs[r].grp_offsets, w_gate, w_up, w_down, bufs[r].h, stream=stream)
+    return [ep_combine_peers(cfg, peers[r], torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=dev),
+                             stream=stream) for r in range(world)]
+
+
+def _barrier(group=None, device=None):
+    """Every rank's earlier work on the current stream is done before any
+    rank's later work starts: a one-element NCCL all-reduce on the stream (no
+    host wait), or a host barrier after the stream drains (gloo)."""
+    if dist.get_backend(group) == "nccl":
+        dist.all_reduce(torch.zeros((1,), dtype=torch.int32, device=device), group=group)
+    else:
+        torch.cuda.current_stream(device).synchronize()
+        dist.barrier(group=group)
+
+
+def gather_table_device(counts, group=None):
+    """table [world, E] int32 on counts' device: row p = counts of rank p."""
+    world = dist.get_world_size(group)
+    if dist.get_backend(group) == "nccl":
+        out = torch.empty((world * counts.numel(),), dtype=counts.dtype, device=counts.device)
+        dist.all_gather_into_tensor(out, counts.contiguous(), group=group)
+        return out.view(world, -1)
+    return torch.from_numpy(gather_table(counts, group).astype(np.int32)).to(counts.device)
+
+
+class EpPeerGroup:
+    """This rank's exchange buffers and the other ranks', mapped into this
+    process: the buffers are exported once (moe_peer_export), the handles are
+    all-gathered, and every other rank's are imported (moe_peer_import).
+    close() releases the mappings; every rank must call it (it ends with a
+    barrier, so that no buffer is freed while another rank still maps it)."""
+
+    def __init__(self, cfg: Config, group=None, device=None):
+        self.cfg, self.group = cfg, group
+        self.rank, self.world = dist.get_rank(group), dist.get_world_size(group)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.device = dev
+        self.bufs = EpPeerBuffers(cfg, self.world, dev)
+        handle = peer_export(self.bufs.raw)
+        handles = [None] * self.world
+        dist.all_gather_object(handles, handle, group=group)
+        self._mapped = []
+        addrs = []
+        for q, hq in enumerate(handles):
+            if q == self.rank:
+                addrs.append(self.bufs.addrs())
+            else:
+                a = peer_import(hq)
+                self._mapped.append((a, hq))
+                addrs.append(self.bufs.addrs(a))
+        self.peers = EpPeers(self.world, self.rank, addrs)
+
+    def close(self):
+        torch.cuda.synchronize(self.device)
+        for a, h in self._mapped:
+            peer_release(a, h)
+        self._mapped = []
+        dist.barrier(group=self.group)
+
+
+def layer_forward_ep_peers(cfg: Config, x, w_router, w_gate, w_up, w_down, logit_bias=None, group=None,
+                           peer_group: EpPeerGroup | None = None, stream=None):
+    """The layer with expert parallelism over peer memory: this rank's tokens
+    in, this rank's output rows out (bit for bit the single-device layer on
+    them).  peer_group: an EpPeerGroup for cfg (made here, and closed, when
+    None)."""
+    own = peer_group is None
+    pg = EpPeerGroup(cfg, group, x.device) if own else peer_group
+    try:
+        # the barriers order the current stream: run every phase on it
+        with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+            disp = ep_route(cfg, x, w_router, logit_bias)
+            table = gather_table_device(disp["counts_kept"], group)
+            ep_dispatch_peers(cfg, pg.peers, table, x, disp, pg.bufs.grp_offsets)
+            _barrier(group, x.device)
+            ep_expert_ffn_peers(cfg, pg.peers, pg.bufs.grp_offsets, w_gate, w_up, w_down, pg.bufs.h)
+            _barrier(group, x.device)
+            return ep_combine_peers(cfg, pg.peers,
+                                    torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=x.device))
+    finally:
+        if own:
+            pg.close()

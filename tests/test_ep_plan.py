@@ -61,3 +61,41 @@ def test_global_capacity_uses_the_whole_batch():
     assert global_capacity(shard, 1200) == int(np.ceil(1.25 * 1200 * 2 / 8))
     inf = Config(300, 256, 384, capacity_factor=float("inf"), dtype="bf16")
     assert global_capacity(inf, 1200) == 1200
+
+
+def test_peer_buffers_layout_is_aligned_and_disjoint():
+    import torch
+
+    from sparse_moe_layer_07_b200 import Config
+    from sparse_moe_layer_07_b200.expert_parallel import EpPeerBuffers
+
+    cfg = Config(300, 256, 384)
+    world = 4
+    b = EpPeerBuffers(cfg, world, "cpu")
+    R = world * cfg.T * cfg.top_k
+    assert b.x_grp.shape == (R, cfg.d) and b.x_grp.dtype == torch.bfloat16
+    assert b.src.numel() == R and b.scale.numel() == R and b.sums.shape == (cfg.T, cfg.d)
+    assert b.h.shape == (R, cfg.f) and b.grp_offsets.numel() == cfg.E + 1
+    parts = [b.x_grp, b.src, b.scale, b.sums]
+    spans = sorted((t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()) for t in parts)
+    for (a0, a1), (b0, _) in zip(spans, spans[1:]):
+        assert a1 <= b0
+    assert spans[-1][1] <= b.raw.data_ptr() + b.raw.numel()
+    # another process sees the same layout from its own mapping of the allocation
+    assert b.addrs() == tuple(t.data_ptr() for t in parts)
+    assert b.addrs(1 << 40) == tuple((1 << 40) + o for o in b.part_offsets)
+    assert all(o % 256 == 0 for o in b.part_offsets)
+
+
+def test_peer_table_checks_its_shape():
+    from sparse_moe_layer_07_b200 import EP_MAX_WORLD, EpPeers
+
+    with pytest.raises(ValueError):
+        EpPeers(EP_MAX_WORLD + 1, 0, [(0, 0, 0, 0)] * (EP_MAX_WORLD + 1))
+    with pytest.raises(ValueError):
+        EpPeers(2, 2, [(0, 0, 0, 0)] * 2)
+    with pytest.raises(ValueError):
+        EpPeers(2, 0, [(0, 0, 0, 0)])
+    p = EpPeers(2, 1, [(16, 32, 48, 64), (80, 96, 112, 128)])
+    assert (p._c.world, p._c.rank) == (2, 1)
+    assert (p._c.x_grp[1], p._c.src[1], p._c.scale[1], p._c.sums[1]) == (80, 96, 112, 128)
