@@ -715,6 +715,8 @@ def main():
                                     args.train_steps)
     if world == 1 and not args.no_configs and w.name == "grok_prefill" and not args.shape and not args.int8:
         line["per_config"] = per_config(moe, W, dev, stream, peaks, peak_src, summ, line.get("decode"))
+    if world == 1 and not args.no_configs and w.name == "grok_prefill" and not args.shape and not args.int8:
+        line["ep_peers"] = ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu and host is not None:
         line["cpu_baseline"] = cpu_baseline(w, host, x_np, args.cpu_tokens)
     if rank == 0:
@@ -835,6 +837,125 @@ def per_config(moe, W_grok, dev, stream, peaks, peak_src, grok_summary, decode):
         out["grok_decode"]["int8_weights"] = {k: decode["int8_weights"][k]
                                               for k in ("ms_per_call", "tokens_per_s", "achieved_gbs", "frac")}
     return out
+
+
+def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, steps=10, warmup=3):
+    """Expert parallelism over peer memory with its `world` ranks held by this
+    process on this GPU: the headline batch split into `world` rank batches of
+    T / world tokens, rank q owning experts [q E / world, (q + 1) E / world).
+    A step runs every rank's routing and dispatch, then every rank's experts,
+    then every rank's rounding on one stream (the stream order stands in for
+    the barriers), so it is the work all `world` GPUs of a real run share,
+    without the NVLink transfers.  The outputs, put back in token order, must
+    equal the single-device layer's on the whole batch bit for bit (no token
+    is dropped at this capacity factor on either side)."""
+    import torch
+
+    from sparse_moe_layer_07_b200.expert_parallel import EpPeerBuffers, ep_route
+
+    Tr = w.T // world
+    cfg = moe.Config(Tr, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16")
+    xs = [x[r * Tr:(r + 1) * Tr] for r in range(world)]
+    bufs = [EpPeerBuffers(cfg, world, dev) for _ in range(world)]
+    addrs = [b.addrs() for b in bufs]
+    peers = [moe.EpPeers(world, r, addrs) for r in range(world)]
+    outs = [torch.empty((Tr, w.d), dtype=torch.bfloat16, device=dev) for _ in range(world)]
+
+    def dispatch_all(disps, table):
+        for r in range(world):
+            moe.ep_dispatch_peers(cfg, peers[r], table, xs[r], disps[r], bufs[r].grp_offsets)
+
+    def step(ev=None):
+        def mark(i):
+            if ev:
+                ev[i].record(stream)
+
+        mark(0)
+        disps = [ep_route(cfg, xs[r], W["wr"], bias_d) for r in range(world)]
+        table = torch.stack([d["counts_kept"] for d in disps])
+        mark(1)
+        dispatch_all(disps, table)
+        mark(2)
+        for r in range(world):
+            moe.ep_expert_ffn_peers(cfg, peers[r], bufs[r].grp_offsets, W["wg"], W["wu"], W["wd"], bufs[r].h)
+        mark(3)
+        for r in range(world):
+            moe.ep_combine_peers(cfg, peers[r], outs[r])
+        mark(4)
+        return disps, table
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        clocks = _sampler(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.monotonic()
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop(window=(w0, time.monotonic()))
+        ms = t0.elapsed_time(t1) / steps
+        # phases on further steps, with events between them
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        phase = [0.0] * 4
+        for i in range(steps):
+            disps, table = step(evs[i])
+            torch.cuda.synchronize(dev)
+            for j in range(4):
+                phase[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / steps
+        n_kept = sum(int(d["offsets"][-1].item()) for d in disps)
+        recv = [int(b.grp_offsets[-1].item()) for b in bufs]
+        single = moe.layer_forward(moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16"), x,
+                                   W["wr"], W["wg"], W["wu"], W["wd"], logit_bias=bias_d)
+        same = bool(torch.equal(torch.cat(outs).view(torch.int16), single.view(torch.int16)))
+        # the dispatch kernels as the GPU runs them: called one by one, each call
+        # spends more time on the host than its kernel on the GPU, so the calls are
+        # captured once in a CUDA graph and replayed back to back (they rewrite the
+        # same rows each time)
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+            dispatch_all(disps, table)
+        torch.cuda.synchronize(dev)
+        stream.wait_stream(cap)
+        for _ in range(3):
+            g.replay()
+        reps = 20
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        disp_ms = g0.elapsed_time(g1) / reps
+        del g
+    device_error = moe.get_device_error()
+    # the dispatch calls: zero the rank's fp32 sums, read each kept row and store
+    # it with its 8 bytes of source id and weight (and read perm, row_scale)
+    dbytes = world * Tr * w.d * 4 + n_kept * (2 * w.d * 2 + 16)
+    dgbs = dbytes / (disp_ms / 1000.0) / 1e9
+    flops = 6.0 * n_kept * w.d * w.f
+    peak, rule = tensor_peak(peaks, peak_src, clk)
+    ex_tf = flops / (phase[2] / 1000.0) / 1e12
+    del bufs, outs
+    return {"world": world, "tokens_per_rank": Tr, "ms_per_step": ms, "tokens_per_s": w.T * 1000.0 / ms,
+            "ms_phases": {"route": phase[0], "dispatch": phase[1], "experts": phase[2], "combine": phase[3]},
+            "dispatch": {"ms": disp_ms, "ms_per_rank": disp_ms / world, "bytes": dbytes, "gbs": dgbs,
+                         "frac_hbm": dgbs / peaks.get("hbm_gbs", 6650.0),
+                         "timing": "the 8 calls (one kernel each) replayed as a CUDA graph, 20 replays"},
+            "experts": {"tflops": ex_tf, "frac": ex_tf / peak, "peak_tflops": peak, "peak_rule": rule},
+            "rows_received": recv, "n_kept": n_kept, "equals_single_device": same, "device_error": device_error,
+            "gpu_launches_per_step": world * 8, "clocks": clk,
+            "phases_timing": "events between the phases of 10 further steps (the short phases include host "
+                             "launch time)",
+            "note": "all ranks on one GPU, one after another: a step is the whole job's work without NVLink; "
+                    "the dispatch stores go to this GPU's own memory here (HBM-bound), to peers' over NVLink "
+                    "in a real run"}
 
 
 def train_bench(moe, cfg, W, x, bias_d, n_kept, dev, stream, peaks, peak_src, world, steps):

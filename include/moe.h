@@ -484,11 +484,15 @@ typedef struct moe_ep_peers_t {
  * (with src and scale) into x_grp of the expert's owner, and writes this rank's
  * grouped offsets as an owner, grp_offsets [E + 1] (experts of other ranks
  * empty).  table [world, E] int32 (device): row p = counts_kept of rank p;
- * offsets, perm, row_scale: this rank's moe_dispatch outputs; x [T, d].  A
- * table row of this rank that disagrees with offsets, or an out-of-range perm
- * entry, sets MOE_DEVERR_OFFSETS / MOE_DEVERR_SLOT_INDEX and stores nothing for
- * the rows concerned.  The stores are fenced at system scope before the kernel
- * ends. */
+ * offsets, perm, row_scale: this rank's moe_dispatch outputs; x [T, d].  One
+ * kernel.  A table inconsistent with offsets (this rank's row differs, a
+ * negative count, more rows for an owner than its buffers hold) sets
+ * MOE_DEVERR_OFFSETS, and the call then stores nothing (sums included) and
+ * writes grp_offsets as all zeros.  An out-of-range perm entry sets
+ * MOE_DEVERR_SLOT_INDEX and skips that row.  The stores (like the adds of
+ * moe_ep_expert_ffn_peers) become visible to the other ranks when the kernel
+ * completes, so the barrier must be ordered after the call on `stream` (a
+ * collective, an event or a host wait), not run concurrently with it. */
 MOE_API moe_status_t moe_ep_dispatch_peers(const moe_config_t* cfg, const moe_ep_peers_t* peers,
                                            const int32_t* table, const void* x, const int32_t* offsets,
                                            const int32_t* perm, const float* row_scale, int32_t* grp_offsets,

@@ -64,96 +64,138 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const uint4* __restrict
   }
 }
 
-// One block per token: routing-weight and logit gradients, then
-// dx[t] = round(dx32[t] + dl_0 W_r[i_0] + dl_1 W_r[i_1]) (slot 0 first).
+// One warp per token: lanes 0 and 1 form the routing-weight gradient of slot
+// 0 / 1 (partials summed in tile order), every lane then has the two logit
+// gradients, lanes 0-7 write the token's dlogits row, and the warp streams
+// dx[t] = round(dx32[t] + dl_0 W_r[i_0] + dl_1 W_r[i_1]) (slot 0 first), four
+// columns per lane and 16-byte vector, four vectors in flight per lane.
 __global__ void __launch_bounds__(256) router_bwd_token_kernel(
     const float* __restrict__ dw_part, int n_parts, const int32_t* __restrict__ slot_of,
     const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, const __nv_bfloat16* __restrict__ wr,
     const float* __restrict__ dx32, int64_t T, int64_t d, int64_t max_slot, float* __restrict__ dlogits,
     float* __restrict__ dweight, __nv_bfloat16* __restrict__ dx, int* err) {
-  __shared__ float s_dl[2];
-  __shared__ int s_e[2];
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    if (threadIdx.x == 0) {
-      float dw[2], w[2];
-      int e[2];
-      for (int j = 0; j < 2; ++j) {
-        int sl = slot_of[2 * t + j];
-        e[j] = topk_idx[2 * t + j];
-        w[j] = topk_w[2 * t + j];
-        if (sl >= max_slot || sl < -1) {
-          flag_error(err, MOE_DEVERR_SLOT_INDEX);
-          sl = -1;
-        }
-        if (e[j] < 0 || e[j] >= kE) {
-          flag_error(err, MOE_DEVERR_EXPERT_INDEX);
-          e[j] = 0;
-          w[j] = 0.f;
-        }
-        float acc = 0.f;
-        if (sl >= 0)
-          for (int p = 0; p < n_parts; ++p) acc += dw_part[(int64_t)sl * n_parts + p];
-        dw[j] = acc;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int nq = (int)(d / 4);  // 4-column groups of a row (d is a multiple of 128)
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    int e = 0;
+    float w = 0.f, dw = 0.f;
+    if (lane < 2) {
+      int sl = slot_of[2 * t + lane];
+      e = topk_idx[2 * t + lane];
+      w = topk_w[2 * t + lane];
+      if (sl >= max_slot || sl < -1) {
+        flag_error(err, MOE_DEVERR_SLOT_INDEX);
+        sl = -1;
       }
-      const float mean = w[0] * dw[0] + w[1] * dw[1];
-      float row[kE];
-      for (int k = 0; k < kE; ++k) row[k] = 0.f;
-      for (int j = 0; j < 2; ++j) {
-        const float dl = w[j] * (dw[j] - mean);
-        row[e[j]] += dl;
-        s_dl[j] = dl;
-        s_e[j] = e[j];
-        dweight[2 * t + j] = dw[j];
+      if (e < 0 || e >= kE) {
+        flag_error(err, MOE_DEVERR_EXPERT_INDEX);
+        e = 0;
+        w = 0.f;
       }
-      for (int k = 0; k < kE; ++k) dlogits[t * kE + k] = row[k];
+      if (sl >= 0)
+        for (int p = 0; p < n_parts; ++p) dw += dw_part[(int64_t)sl * n_parts + p];
+      dweight[2 * t + lane] = dw;
     }
-    __syncthreads();
-    const float dl0 = s_dl[0], dl1 = s_dl[1];
-    const __nv_bfloat16* w0 = wr + (int64_t)s_e[0] * d;
-    const __nv_bfloat16* w1 = wr + (int64_t)s_e[1] * d;
-    for (int64_t i = 2 * (int64_t)threadIdx.x; i < d; i += 2 * (int64_t)blockDim.x) {
-      const float2 a = *reinterpret_cast<const float2*>(dx32 + t * d + i);
-      const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(w0 + i));
-      const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(w1 + i));
-      float v0 = a.x + dl0 * p.x;
-      float v1 = a.y + dl0 * p.y;
-      v0 = v0 + dl1 * q.x;
-      v1 = v1 + dl1 * q.y;
-      *reinterpret_cast<uint32_t*>(dx + t * d + i) = pack_bf16x2(v0, v1);
+    const int e0 = __shfl_sync(0xffffffffu, e, 0), e1 = __shfl_sync(0xffffffffu, e, 1);
+    const float w0 = __shfl_sync(0xffffffffu, w, 0), w1 = __shfl_sync(0xffffffffu, w, 1);
+    const float dw0 = __shfl_sync(0xffffffffu, dw, 0), dw1 = __shfl_sync(0xffffffffu, dw, 1);
+    const float mean = w0 * dw0 + w1 * dw1;
+    const float dl0 = w0 * (dw0 - mean);
+    const float dl1 = w1 * (dw1 - mean);
+    if (lane < kE) {
+      float v = 0.f;
+      if (e0 == lane) v += dl0;
+      if (e1 == lane) v += dl1;
+      dlogits[t * kE + lane] = v;
     }
-    __syncthreads();  // s_dl / s_e are rewritten for the next token
+    const float4* a4 = reinterpret_cast<const float4*>(dx32 + t * d);
+    const uint2* p2 = reinterpret_cast<const uint2*>(wr + (int64_t)e0 * d);
+    const uint2* q2 = reinterpret_cast<const uint2*>(wr + (int64_t)e1 * d);
+    uint2* o2 = reinterpret_cast<uint2*>(dx + t * d);
+    for (int g0 = lane; g0 < nq; g0 += 128) {
+      float4 a[4];
+      uint2 pb[4], qb[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int g = g0 + 32 * k;
+        if (g < nq) {
+          a[k] = __ldcs(a4 + g);
+          pb[k] = p2[g];
+          qb[k] = q2[g];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int g = g0 + 32 * k;
+        if (g < nq) {
+          const float2 p01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pb[k].x));
+          const float2 p23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pb[k].y));
+          const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qb[k].x));
+          const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qb[k].y));
+          float v0 = a[k].x + dl0 * p01.x, v1 = a[k].y + dl0 * p01.y;
+          float v2 = a[k].z + dl0 * p23.x, v3 = a[k].w + dl0 * p23.y;
+          v0 = v0 + dl1 * q01.x;
+          v1 = v1 + dl1 * q01.y;
+          v2 = v2 + dl1 * q23.x;
+          v3 = v3 + dl1 * q23.y;
+          o2[g] = make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
+        }
+      }
+    }
   }
 }
 
 // dW_r partial sums over token chunks: part[c][e][i] = sum_{t in chunk c} dlogits[t, e] x[t, i]
-// (tokens in increasing order), one thread per column i.
+// (tokens in increasing order); a thread owns 8 adjacent columns (one 16-byte
+// vector of x per token) for all 8 experts, and keeps two tokens' loads in flight.
 __global__ void __launch_bounds__(256) router_bwd_weight_kernel(const float* __restrict__ dlogits,
                                                                const __nv_bfloat16* __restrict__ x, int64_t T,
                                                                int64_t d, int chunks, float* __restrict__ part) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
   const int c = blockIdx.y;
   const int64_t per = (T + chunks - 1) / chunks;
   const int64_t t0 = c * per;
   const int64_t t1 = t0 + per < T ? t0 + per : T;
-  if (i >= d) return;
-  float acc[kE];
+  const int64_t nv = d / 8;
+  if (v >= nv) return;
+  float acc[kE][8];
 #pragma unroll
-  for (int e = 0; e < kE; ++e) acc[e] = 0.f;
-  for (int64_t t = t0; t < t1; ++t) {
-    const float xv = __bfloat162float(x[t * d + i]);
-    const float4 l0 = *reinterpret_cast<const float4*>(dlogits + t * kE);
-    const float4 l1 = *reinterpret_cast<const float4*>(dlogits + t * kE + 4);
-    acc[0] = fmaf(l0.x, xv, acc[0]);
-    acc[1] = fmaf(l0.y, xv, acc[1]);
-    acc[2] = fmaf(l0.z, xv, acc[2]);
-    acc[3] = fmaf(l0.w, xv, acc[3]);
-    acc[4] = fmaf(l1.x, xv, acc[4]);
-    acc[5] = fmaf(l1.y, xv, acc[5]);
-    acc[6] = fmaf(l1.z, xv, acc[6]);
-    acc[7] = fmaf(l1.w, xv, acc[7]);
+  for (int e = 0; e < kE; ++e)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[e][k] = 0.f;
+  const uint4* x4 = reinterpret_cast<const uint4*>(x);
+  int64_t t = t0;
+  for (; t + 1 < t1; t += 2) {
+    const uint4 qa = __ldcs(x4 + t * nv + v);
+    const uint4 qb = __ldcs(x4 + (t + 1) * nv + v);
+    float xa[8], xb[8];
+    unpack8(qa, xa);
+    unpack8(qb, xb);
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+      const float la = __ldg(dlogits + t * kE + e);
+      const float lb = __ldg(dlogits + (t + 1) * kE + e);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[e][k] = fmaf(lb, xb[k], fmaf(la, xa[k], acc[e][k]));
+    }
+  }
+  if (t < t1) {
+    float xa[8];
+    unpack8(__ldcs(x4 + t * nv + v), xa);
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+      const float la = __ldg(dlogits + t * kE + e);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[e][k] = fmaf(la, xa[k], acc[e][k]);
+    }
   }
 #pragma unroll
-  for (int e = 0; e < kE; ++e) part[((int64_t)c * kE + e) * d + i] = acc[e];
+  for (int e = 0; e < kE; ++e) {
+    float4* o = reinterpret_cast<float4*>(part + ((int64_t)c * kE + e) * d + v * 8);
+    o[0] = make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
+    o[1] = make_float4(acc[e][4], acc[e][5], acc[e][6], acc[e][7]);
+  }
 }
 
 // dW_r[e][i] = sum over chunks in order; block 0 also forms dbias[e] = sum_t dlogits[t, e]
@@ -210,12 +252,12 @@ cudaError_t launch_router_bwd(const moe_config_t& c, const float* dw_part, int n
                               const void* x, float* dlogits, float* dweight, void* dx, float* dw_router,
                               float* dbias, float* wr_part, cudaStream_t s, const Ctx& ctx) {
   if (c.T == 0) return cudaSuccess;
-  router_bwd_token_kernel<<<capped(c.T, ctx), 256, 0, s>>>(
+  router_bwd_token_kernel<<<capped((c.T + 7) / 8, ctx), 256, 0, s>>>(
       dw_part, n_parts, slot_of, topk_idx, topk_w, static_cast<const __nv_bfloat16*>(w_router), dx32, c.T, c.d,
       slot_rows(c), dlogits, dweight, static_cast<__nv_bfloat16*>(dx), ctx.err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((c.d + 255) / 256), (unsigned)kRouterBwdChunks);
+  dim3 grid((unsigned)((c.d / 8 + 255) / 256), (unsigned)kRouterBwdChunks);
   router_bwd_weight_kernel<<<grid, 256, 0, s>>>(dlogits, static_cast<const __nv_bfloat16*>(x), c.T, c.d,
                                                 kRouterBwdChunks, wr_part);
   e = cudaGetLastError();

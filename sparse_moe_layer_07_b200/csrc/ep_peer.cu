@@ -11,6 +11,8 @@
 //             fused combine epilogue) adds routing_weight * (h W_down) into the
 //             source rank's fp32 sums with vector atomics; the source then
 //             rounds its own sums once.
+// Neither kernel signals another rank: the phases are separated by barriers
+// the caller puts after them on the stream.
 // Within an owner's buffer, expert e's rows come from source 0, 1, ... in
 // turn, each source's rows in its kept (token) order, so every rank computes
 // every destination from the all-gathered table of kept counts alone.
@@ -38,6 +40,7 @@ struct EpDispatchArgs {
   int32_t* grp_offsets;     // [E + 1] out: this rank's received rows by expert
   int64_t T;                // tokens of every rank
   int64_t rows_cap;         // rows of every grouped buffer: world * T * top_k
+  float* sums;              // this rank's fp32 sums [T, d], cleared here
   int row_vec;
   int world, rank;
   uint4* x_grp[MOE_EP_MAX_WORLD];
@@ -76,85 +79,103 @@ __device__ __forceinline__ float* scale_select(const EpDispatchArgs& a, int q) {
   return d;
 }
 
-// One warp per kept row (grid-stride).  Every block derives the destinations
-// from the table in shared memory: dst[e] = first row, in the owner's buffer,
-// of this rank's rows of expert e = (rows of the owner's earlier experts, all
-// sources) + (rows of expert e from sources before this rank).
+// Work items of one warp: a 2 KB segment of a kept row (32 lanes x 4 vectors
+// of 16 bytes) to copy into its owner's buffer, or, after all of those, 2 KB
+// of this rank's fp32 sums to clear.  Every block first derives, one thread per
+// expert, dst[e] = first row in the owner's buffer of this rank's rows of
+// expert e = (rows of the owner's earlier experts, from every source) + (rows
+// of expert e from sources before this rank), and checks the table.
+constexpr int kSegVec = 128;  // 16-byte vectors per work item
+
 __global__ void __launch_bounds__(32 * kWarps) ep_dispatch_peers_kernel(const __grid_constant__ EpDispatchArgs a) {
   __shared__ int s_offs[kE + 1];
   __shared__ int s_dst[kE];
-  __shared__ int s_ok;
   pdl_wait();
-  if (threadIdx.x == 0) {
-    const int per = kE / a.world;
-    bool ok = true;
-    for (int e = 0; e <= kE; ++e) s_offs[e] = __ldg(a.offsets + e);
-    if (s_offs[0] != 0) ok = false;
-    for (int e = 0; e < kE; ++e)
-      if (s_offs[e + 1] - s_offs[e] != __ldg(a.table + a.rank * kE + e)) ok = false;
-    if (s_offs[kE] > a.T * 2) ok = false;
-    for (int q = 0; q < a.world; ++q) {
-      int64_t pos = 0;
-      for (int e = q * per; e < (q + 1) * per; ++e)
-        for (int p = 0; p < a.world; ++p) {
-          const int c = __ldg(a.table + p * kE + e);
-          if (c < 0) ok = false;
-          if (p == a.rank) s_dst[e] = (int)pos;
-          pos += c;
-        }
-      if (pos > a.rows_cap) ok = false;
-    }
-    if (blockIdx.x == 0) {
-      // this rank as an owner: its experts in order, other experts empty
-      int run = 0;
-      for (int e = 0; e < kE; ++e) {
-        a.grp_offsets[e] = ok ? run : 0;
-        if (e / per == a.rank)
-          for (int p = 0; p < a.world; ++p) run += __ldg(a.table + p * kE + e);
-      }
-      a.grp_offsets[kE] = ok ? run : 0;
-      if (!ok) flag_error(a.err, MOE_DEVERR_OFFSETS);
-    }
-    s_ok = ok;
-  }
-  __syncthreads();
-  if (!s_ok) return;
   const int per = kE / a.world;
+  if (threadIdx.x <= kE) s_offs[threadIdx.x] = __ldg(a.offsets + threadIdx.x);
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x < kE) {
+    const int e = threadIdx.x;
+    const int q = e / per;
+    if (s_offs[e + 1] - s_offs[e] != __ldg(a.table + a.rank * kE + e)) ok = false;
+    int64_t pos = 0, total = 0;
+    for (int e2 = q * per; e2 < (q + 1) * per; ++e2)
+      for (int p = 0; p < a.world; ++p) {
+        const int c = __ldg(a.table + p * kE + e2);
+        if (c < 0) ok = false;
+        if (e2 < e || (e2 == e && p < a.rank)) pos += c;
+        total += c;
+      }
+    if (total > a.rows_cap) ok = false;
+    s_dst[e] = (int)pos;
+  }
+  if (threadIdx.x == 0 && (s_offs[0] != 0 || s_offs[kE] > a.T * 2)) ok = false;
+  ok = __syncthreads_and(ok);
+  if (blockIdx.x == 0 && threadIdx.x <= kE) {
+    // this rank as an owner: its experts in order, other experts empty
+    int run = 0;
+    for (int e2 = a.rank * per; e2 < (a.rank + 1) * per && e2 < (int)threadIdx.x; ++e2)
+      for (int p = 0; p < a.world; ++p) run += __ldg(a.table + p * kE + e2);
+    a.grp_offsets[threadIdx.x] = ok ? run : 0;
+    if (!ok && threadIdx.x == 0) flag_error(a.err, MOE_DEVERR_OFFSETS);
+  }
+  if (!ok) return;
   const int lane = threadIdx.x & 31;
   const int n = s_offs[kE];
   const int nv = a.row_vec;
-  for (int r = blockIdx.x * kWarps + (threadIdx.x >> 5); r < n; r += gridDim.x * kWarps) {
-    int e = 0;
+  const int segs = (nv + kSegVec - 1) / kSegVec;
+  const int64_t copy_items = (int64_t)n * segs;
+  const int64_t zero_vec = a.T * (int64_t)nv * 2;  // the sums hold T rows of 4 * d bytes
+  const int64_t items = copy_items + (zero_vec + kSegVec - 1) / kSegVec;
+  const int64_t warps = (int64_t)gridDim.x * kWarps;
+  for (int64_t it = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); it < items; it += warps) {
+    if (it < copy_items) {
+      const int r = (int)(it / segs);
+      const int v0 = (int)(it - (int64_t)r * segs) * kSegVec;
+      int e = 0;
 #pragma unroll
-    for (int k = 1; k < kE; ++k)
-      if (r >= s_offs[k]) e = k;
-    const int q = e / per;
-    const int64_t dst = (int64_t)s_dst[e] + (r - s_offs[e]);
-    const int t = __ldg(a.perm + r);
-    if (t < 0 || (int64_t)t >= a.T) {
-      if (lane == 0) flag_error(a.err, MOE_DEVERR_SLOT_INDEX);
-      continue;
-    }
-    const uint4* srow = a.x + (int64_t)t * nv;
-    uint4* drow = peer_select(a, q) + dst * nv;
-    // four 16-byte loads in flight per lane before the stores
-    for (int i = lane; i < nv; i += 128) {
+      for (int k = 1; k < kE; ++k)
+        if (r >= s_offs[k]) e = k;
+      const int q = e / per;
+      const int64_t dst = (int64_t)s_dst[e] + (r - s_offs[e]);
+      const int t = __ldg(a.perm + r);
+      if (t < 0 || (int64_t)t >= a.T) {
+        if (lane == 0) flag_error(a.err, MOE_DEVERR_SLOT_INDEX);
+        continue;
+      }
+      const uint4* srow = a.x + (int64_t)t * nv;
+      uint4* drow = peer_select(a, q) + dst * nv;
       uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (i + 32 * j < nv) v[j] = ld_stream(srow + i + 32 * j);
+      for (int j = 0; j < 4; ++j) {
+        const int i = v0 + lane + 32 * j;
+        if (i < nv) v[j] = ld_stream(srow + i);
+      }
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (i + 32 * j < nv) drow[i + 32 * j] = v[j];
-    }
-    if (lane == 0) {
-      src_select(a, q)[dst] = (int32_t)(a.rank * a.T + t);
-      scale_select(a, q)[dst] = __ldg(a.row_scale + r);
+      for (int j = 0; j < 4; ++j) {
+        const int i = v0 + lane + 32 * j;
+        if (i < nv) drow[i] = v[j];
+      }
+      if (v0 == 0 && lane == 0) {
+        src_select(a, q)[dst] = (int32_t)(a.rank * a.T + t);
+        scale_select(a, q)[dst] = __ldg(a.row_scale + r);
+      }
+    } else {
+      const int64_t z0 = (it - copy_items) * kSegVec;
+      uint4* z = reinterpret_cast<uint4*>(a.sums);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t i = z0 + lane + 32 * j;
+        if (i < zero_vec) z[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
-  // the stores reach other GPUs' memory: make them visible system-wide before
-  // whatever the caller uses as the barrier can signal the owners
-  __threadfence_system();
+  // No fence: the owners read these rows only after a barrier that the caller
+  // orders after this kernel on the stream (a collective, an event or a host
+  // barrier), and a kernel's completion makes all its stores, peer memory
+  // included, visible.  A fence per block cost 6 us of 25 at 75 MB per rank
+  // (one per thread: 11 us).
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -209,9 +230,8 @@ extern "C" moe_status_t moe_ep_dispatch_peers(const moe_config_t* cfg, const moe
   Ctx ctx;
   if ((st = current_ctx(ctx)) != MOE_OK) return st;
   const int r = peers->rank;
-  cudaError_t e = launch_zero_rows(*cfg, peers->sums[r], stream, ctx);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
   EpDispatchArgs a = {};
+  a.sums = peers->sums[r];
   a.x = static_cast<const uint4*>(x);
   a.table = table;
   a.offsets = offsets;
@@ -229,11 +249,14 @@ extern "C" moe_status_t moe_ep_dispatch_peers(const moe_config_t* cfg, const moe
     a.scale[q] = peers->scale[q];
   }
   a.err = ctx.err;
-  // one warp per row: enough blocks for every row up to 8 blocks per SM
-  int64_t blocks = (slot_rows(*cfg) + kWarps - 1) / kWarps;
+  // one warp per 2 KB item: enough blocks for the most items (every row kept)
+  // up to 8 blocks per SM
+  const int64_t segs = (a.row_vec + kSegVec - 1) / kSegVec;
+  const int64_t items = slot_rows(*cfg) * segs + (cfg->T * (int64_t)a.row_vec * 2 + kSegVec - 1) / kSegVec;
+  int64_t blocks = (items + kWarps - 1) / kWarps;
   if (blocks > (int64_t)ctx.num_sms * 8) blocks = (int64_t)ctx.num_sms * 8;
   if (blocks < 1) blocks = 1;
-  e = launch_pdl(ep_dispatch_peers_kernel, dim3((unsigned)blocks), dim3(32 * kWarps), 0, stream, no_extra_attr(), a);
+  cudaError_t e = launch_pdl(ep_dispatch_peers_kernel, dim3((unsigned)blocks), dim3(32 * kWarps), 0, stream, no_extra_attr(), a);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -425,8 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
-    // adds into other GPUs' memory: visible system-wide before the kernel ends
-    if (kScatter && args.n_peers > 0) __threadfence_system();
   }
 
   __syncthreads();
@@ -659,7 +657,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * buf);
     }
-    if (kScatter && args.n_peers > 0) __threadfence_system();
   }
 
   __syncthreads();

@@ -164,7 +164,7 @@ cudaError_t launch_router_bwd(const moe_config_t& c, const float* dw_part, int n
                               const int32_t* topk_idx, const float* topk_w, const void* w_router, const float* dx32,
                               const void* x, float* dlogits, float* dweight, void* dx, float* dw_router,
                               float* dbias, float* wr_part, cudaStream_t s, const Ctx& ctx);
-constexpr int kRouterBwdChunks = 32;  // token chunks of the dW_r partial sums
+constexpr int kRouterBwdChunks = 128;  // token chunks of the dW_r partial sums
 
 // out32 <- 0 ([T, d] fp32), and out <- out32 rounded to cfg's dtype.
 cudaError_t launch_zero_rows(const moe_config_t& c, float* out32, cudaStream_t s, const Ctx& ctx);
