@@ -625,6 +625,8 @@ def main():
                     help="tile shape of the bf16 grouped GEMMs")
     ap.add_argument("--unfused", action="store_true",
                     help="separate down and combine kernels instead of the fused down-combine")
+    ap.add_argument("--ep-only", action="store_true",
+                    help="only the expert-parallel measurement (8 ranks on this GPU), e.g. for profiling its kernels")
     args = ap.parse_args()
     w = configs.WORKLOADS[args.workload]
     if args.shape:
@@ -665,6 +667,13 @@ def main():
     bias = configs.make_bias(w)
     bias_d = None if bias is None else to_dev(bias, dev)
     stream = torch.cuda.current_stream(dev)
+    if args.ep_only:
+        if world > 1 or w.storage != "bf16" or w.T % 8 or w.d % 256:
+            raise SystemExit("--ep-only: one GPU, a bf16 workload, T a multiple of 8 and d of 256")
+        peaks, peak_src = load_peaks()
+        print(json.dumps({"workload": w.name, "ep_peers": ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks,
+                                                                          peak_src)}), flush=True)
+        return
     run = LayerRun(moe, w, W, x, bias_d, dev, stream, int8=args.int8, unfused=args.unfused)
     cfg, tdt = run.cfg, run.cfg.torch_dtype
     res = run.time(args.steps, args.warmup, world)

@@ -90,19 +90,25 @@ constexpr int kSegVec = 128;  // 16-byte vectors per work item
 __global__ void __launch_bounds__(32 * kWarps) ep_dispatch_peers_kernel(const __grid_constant__ EpDispatchArgs a) {
   __shared__ int s_offs[kE + 1];
   __shared__ int s_dst[kE];
+  __shared__ int s_tab[MOE_EP_MAX_WORLD * kE];
   pdl_wait();
   const int per = kE / a.world;
+  // one round of loads: the offsets (threads 0-8) and the table (threads 32-95);
+  // at 75 MB per call the kernel is latency-bound, and a second dependent round
+  // cost 4 us of 18 (a grid of one resident wave, 4 us more: the extra blocks
+  // hide latency better than they cost in prologues)
   if (threadIdx.x <= kE) s_offs[threadIdx.x] = __ldg(a.offsets + threadIdx.x);
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + a.world * kE) s_tab[threadIdx.x - 32] = __ldg(a.table + threadIdx.x - 32);
   __syncthreads();
   bool ok = true;
   if (threadIdx.x < kE) {
     const int e = threadIdx.x;
     const int q = e / per;
-    if (s_offs[e + 1] - s_offs[e] != __ldg(a.table + a.rank * kE + e)) ok = false;
+    if (s_offs[e + 1] - s_offs[e] != s_tab[a.rank * kE + e]) ok = false;
     int64_t pos = 0, total = 0;
     for (int e2 = q * per; e2 < (q + 1) * per; ++e2)
       for (int p = 0; p < a.world; ++p) {
-        const int c = __ldg(a.table + p * kE + e2);
+        const int c = s_tab[p * kE + e2];
         if (c < 0) ok = false;
         if (e2 < e || (e2 == e && p < a.rank)) pos += c;
         total += c;
@@ -116,7 +122,7 @@ __global__ void __launch_bounds__(32 * kWarps) ep_dispatch_peers_kernel(const __
     // this rank as an owner: its experts in order, other experts empty
     int run = 0;
     for (int e2 = a.rank * per; e2 < (a.rank + 1) * per && e2 < (int)threadIdx.x; ++e2)
-      for (int p = 0; p < a.world; ++p) run += __ldg(a.table + p * kE + e2);
+      for (int p = 0; p < a.world; ++p) run += s_tab[p * kE + e2];
     a.grp_offsets[threadIdx.x] = ok ? run : 0;
     if (!ok && threadIdx.x == 0) flag_error(a.err, MOE_DEVERR_OFFSETS);
   }
