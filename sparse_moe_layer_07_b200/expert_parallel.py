@@ -218,14 +218,15 @@ def ep_forward_peers_local(cfg: Config, xs, w_router, w_gate, w_up, w_down, logi
                              stream=stream) for r in range(world)]
 
 
-def _barrier(group=None, device=None):
+def ep_barrier(group=None, device=None):
     """Every rank's earlier work on the current stream is done before any
     rank's later work starts: a one-element NCCL all-reduce on the stream (no
     host wait), or a host barrier after the stream drains (gloo)."""
     if dist.get_backend(group) == "nccl":
         dist.all_reduce(torch.zeros((1,), dtype=torch.int32, device=device), group=group)
     else:
-        torch.cuda.current_stream(device).synchronize()
+        if device is not None and torch.device(device).type == "cuda":
+            torch.cuda.current_stream(device).synchronize()
         dist.barrier(group=group)
 
 
@@ -288,9 +289,9 @@ def layer_forward_ep_peers(cfg: Config, x, w_router, w_gate, w_up, w_down, logit
             disp = ep_route(cfg, x, w_router, logit_bias)
             table = gather_table_device(disp["counts_kept"], group)
             ep_dispatch_peers(cfg, pg.peers, table, x, disp, pg.bufs.grp_offsets)
-            _barrier(group, x.device)
+            ep_barrier(group, x.device)
             ep_expert_ffn_peers(cfg, pg.peers, pg.bufs.grp_offsets, w_gate, w_up, w_down, pg.bufs.h)
-            _barrier(group, x.device)
+            ep_barrier(group, x.device)
             return ep_combine_peers(cfg, pg.peers,
                                     torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=x.device))
     finally:

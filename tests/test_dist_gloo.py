@@ -137,13 +137,18 @@ def _ep_worker(rank, world, port, q):
 
     sys.path.insert(0, ROOT)
     import oracle
-    from sparse_moe_layer_07_b200.expert_parallel import _all_to_all_rows, ep_plan, gather_table
+    from sparse_moe_layer_07_b200.expert_parallel import (_all_to_all_rows, ep_barrier, ep_plan, gather_table,
+                                                          gather_table_device)
 
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
         idx, w, cap, per = _ep_routing(oracle, world, rank)
         disp = oracle.dispatch(idx, w, 8, cap)
         table = gather_table(torch.from_numpy(disp["counts_kept"].astype(np.int32)))
+        # the peer-memory path's table (int32 tensor on the counts' device) and barrier
+        t_dev = gather_table_device(torch.from_numpy(disp["counts_kept"].astype(np.int32)))
+        assert t_dev.dtype == torch.int32 and np.array_equal(t_dev.numpy(), table)
+        ep_barrier(device="cpu")
         plan = ep_plan(table, rank, world)
         # each row carries (source rank, token, expert)
         n = disp["n_kept"]
