@@ -258,13 +258,20 @@ class EpPeerGroup:
         dist.all_gather_object(handles, handle, group=group)
         self._mapped = []
         addrs = []
-        for q, hq in enumerate(handles):
-            if q == self.rank:
-                addrs.append(self.bufs.addrs())
-            else:
-                a = peer_import(hq)
-                self._mapped.append((a, hq))
-                addrs.append(self.bufs.addrs(a))
+        try:
+            for q, hq in enumerate(handles):
+                if q == self.rank:
+                    addrs.append(self.bufs.addrs())
+                else:
+                    a = peer_import(hq)
+                    self._mapped.append((a, hq))
+                    addrs.append(self.bufs.addrs(a))
+        except Exception:
+            # leave nothing mapped; the other ranks learn of it at their next collective
+            for a, h in self._mapped:
+                peer_release(a, h)
+            self._mapped = []
+            raise
         self.peers = EpPeers(self.world, self.rank, addrs)
 
     def close(self):
