@@ -848,7 +848,8 @@ def per_config(moe, W_grok, dev, stream, peaks, peak_src, grok_summary, decode):
     return out
 
 
-def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, steps=10, warmup=3):
+def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, steps=100, warmup=3,
+                   phase_steps=10):
     """Expert parallelism over peer memory with its `world` ranks held by this
     process on this GPU: the headline batch split into `world` rank batches of
     T / world tokens, rank q owning experts [q E / world, (q + 1) E / world).
@@ -857,7 +858,8 @@ def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, 
     the barriers), so it is the work all `world` GPUs of a real run share,
     without the NVLink transfers.  The outputs, put back in token order, must
     equal the single-device layer's on the whole batch bit for bit (no token
-    is dropped at this capacity factor on either side)."""
+    is dropped at this capacity factor on either side).  `steps` matches the
+    headline's timed steps so that both run under the same power-capped clock."""
     import torch
 
     from sparse_moe_layer_07_b200.expert_parallel import EpPeerBuffers, ep_route
@@ -908,13 +910,13 @@ def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, 
         clk = clocks.stop(window=(w0, time.monotonic()))
         ms = t0.elapsed_time(t1) / steps
         # phases on further steps, with events between them
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(phase_steps)]
         phase = [0.0] * 4
-        for i in range(steps):
+        for i in range(phase_steps):
             disps, table = step(evs[i])
             torch.cuda.synchronize(dev)
             for j in range(4):
-                phase[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / steps
+                phase[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / phase_steps
         n_kept = sum(int(d["offsets"][-1].item()) for d in disps)
         recv = [int(b.grp_offsets[-1].item()) for b in bufs]
         single = moe.layer_forward(moe.Config(w.T, w.d, w.f, capacity_factor=w.capacity_factor, dtype="bf16"), x,
@@ -952,7 +954,8 @@ def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, 
     peak, rule = tensor_peak(peaks, peak_src, clk)
     ex_tf = flops / (phase[2] / 1000.0) / 1e12
     del bufs, outs
-    return {"world": world, "tokens_per_rank": Tr, "ms_per_step": ms, "tokens_per_s": w.T * 1000.0 / ms,
+    return {"world": world, "tokens_per_rank": Tr, "steps": steps, "ms_per_step": ms,
+            "tokens_per_s": w.T * 1000.0 / ms,
             "ms_phases": {"route": phase[0], "dispatch": phase[1], "experts": phase[2], "combine": phase[3]},
             "dispatch": {"ms": disp_ms, "ms_per_rank": disp_ms / world, "bytes": dbytes, "gbs": dgbs,
                          "frac_hbm": dgbs / peaks.get("hbm_gbs", 6650.0),
@@ -960,8 +963,8 @@ def ep_peers_bench(moe, w, W, x, bias_d, dev, stream, peaks, peak_src, world=8, 
             "experts": {"tflops": ex_tf, "frac": ex_tf / peak, "peak_tflops": peak, "peak_rule": rule},
             "rows_received": recv, "n_kept": n_kept, "equals_single_device": same, "device_error": device_error,
             "gpu_launches_per_step": world * 8, "clocks": clk,
-            "phases_timing": "events between the phases of 10 further steps (the short phases include host "
-                             "launch time)",
+            "phases_timing": f"events between the phases of {phase_steps} further steps (the short phases "
+                             "include host launch time)",
             "note": "all ranks on one GPU, one after another: a step is the whole job's work without NVLink; "
                     "the dispatch stores go to this GPU's own memory here (HBM-bound), to peers' over NVLink "
                     "in a real run"}
