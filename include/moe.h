@@ -469,7 +469,9 @@ MOE_API moe_status_t moe_profile_read(float* ms, int32_t* calls, int32_t n);
  * in the fused down + combine scope (bf16, d a multiple of 256, top_k 2; every
  * row's products and its two-term fp32 sum do not depend on which rows share a
  * tile or on the order of the two adds).  world in {1, 2, 4, 8} (dividing E =
- * 8) and world * T <= 2^30, else MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG. */
+ * 8) and world * T <= 2^30, else MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG;
+ * x_grp and sums 16-byte aligned, src and scale 4-byte aligned, none NULL for
+ * q < world (MOE_ERR_INVALID_ARG). */
 #define MOE_EP_MAX_WORLD 8
 typedef struct moe_ep_peers_t {
   int32_t world;

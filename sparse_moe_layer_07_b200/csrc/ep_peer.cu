@@ -199,7 +199,8 @@ moe_status_t check_ep(const moe_config_t* cfg, const moe_ep_peers_t* peers) {
   if ((int64_t)w * cfg->T > ((int64_t)1 << 30)) return MOE_ERR_INVALID_ARG;
   for (int q = 0; q < w; ++q)
     if (!peers->x_grp[q] || !peers->src[q] || !peers->scale[q] || !peers->sums[q] || !aligned16(peers->x_grp[q]) ||
-        !aligned16(peers->sums[q]))
+        !aligned16(peers->sums[q]) || (reinterpret_cast<uintptr_t>(peers->src[q]) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(peers->scale[q]) & 3u) != 0)
       return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }

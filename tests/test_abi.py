@@ -276,3 +276,40 @@ def test_phase_profile_read_without_events(moe):
         assert moe.lib.moe_profile_read(ms, calls, -1) == 1
     finally:
         moe.profile_phases(False)
+
+
+def test_peer_entry_points_check_arguments_before_any_cuda_call():
+    # every case below is rejected on the host before the library touches CUDA,
+    # so fake device addresses are never dereferenced
+    import ctypes
+
+    from sparse_moe_layer_07_b200 import Config, EpPeers, lib
+
+    cfg = Config(512, 256, 384)
+    good = [(0x10000 * (q + 1), 0x100000 + 0x1000 * q, 0x200000 + 0x1000 * q, 0x300000 + 0x1000 * q)
+            for q in range(2)]
+    fake = ctypes.c_void_p(0x400000)
+
+    def dispatch(peers, c=cfg):
+        return lib.moe_ep_dispatch_peers(c.ref, peers.ref, fake, fake, fake, fake, fake, fake, None)
+
+    def ffn(peers, c=cfg):
+        return lib.moe_ep_expert_ffn_peers(c.ref, peers.ref, fake, fake, fake, fake, fake, None)
+
+    def combine(peers, c=cfg):
+        return lib.moe_ep_combine_peers(c.ref, peers.ref, fake, None)
+
+    def with_part(q, k, delta):
+        rows = [list(r) for r in good]
+        rows[q][k] += delta
+        return EpPeers(2, 0, [tuple(r) for r in rows])
+
+    for call in (dispatch, ffn, combine):
+        assert call(with_part(1, 1, 2)) == 1      # src not 4-byte aligned
+        assert call(with_part(0, 2, 1)) == 1      # scale not 4-byte aligned
+        assert call(with_part(1, 0, 8)) == 1      # x_grp not 16-byte aligned
+        assert call(with_part(0, 3, 4)) == 1      # sums not 16-byte aligned
+        assert call(with_part(1, 3, -good[1][3])) == 1  # a NULL buffer
+        assert call(EpPeers(3, 0, good + [good[0]])) == 2  # 3 ranks do not divide E = 8
+        assert call(EpPeers(2, 0, good), Config(512, 256, 384, dtype="f32")) == 2
+        assert call(EpPeers(2, 0, good), Config(512, 128, 384)) == 2  # d not a multiple of 256
