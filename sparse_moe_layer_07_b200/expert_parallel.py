@@ -275,7 +275,8 @@ class EpPeerGroup:
         self.peers = EpPeers(self.world, self.rank, addrs)
 
     def close(self):
-        torch.cuda.synchronize(self.device)
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
         for a, h in self._mapped:
             peer_release(a, h)
         self._mapped = []

@@ -210,3 +210,83 @@ def test_expert_parallel_exchange_on_gloo_ranks(world):
         assert all(offsets[e + 1] == offsets[e] for e in range(8) if e // n_own != rank)
         # the return trip puts every row back where this rank sent it from
         assert np.array_equal(back, sent[:back.shape[0]]) and back.shape[0] == sent.shape[0]
+
+
+def _peer_group_worker(rank, world, port, q, fail_rank):
+    # EpPeerGroup's mapping lifecycle on gloo ranks, with the CUDA IPC calls
+    # replaced by host fakes (no GPU): handles are exchanged, every other
+    # rank's buffers are "imported", close() releases each mapping once, and
+    # an import that fails releases what was already mapped before raising
+    import sys
+
+    sys.path.insert(0, ROOT)
+    from sparse_moe_layer_07_b200 import Config
+    import sparse_moe_layer_07_b200.expert_parallel as ep
+
+    released = []
+    ep.peer_export = lambda t: f"handle-{rank}".encode()
+
+    def fake_import(h):
+        src = int(h.decode().split("-")[1])
+        if rank == fail_rank and src == world - 1:
+            raise RuntimeError("import refused")
+        return (1 << 40) * (src + 1)
+
+    ep.peer_import = fake_import
+    ep.peer_release = lambda addr, h: released.append((addr, h))
+    from datetime import timedelta
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=10))
+    try:
+        cfg = Config(64, 256, 384)
+        try:
+            pg = ep.EpPeerGroup(cfg, device="cpu")
+        except RuntimeError as exc:
+            q.put((rank, "raised", str(exc), released))
+            return
+        addrs = [tuple(pg.peers._c.x_grp[i] for i in range(world)), tuple(pg.peers._c.sums[i] for i in range(world))]
+        own = pg.bufs.addrs()
+        try:
+            pg.close()
+            status = "ok"
+        except RuntimeError:
+            # a rank that failed never reaches close()'s barrier: the others see it fail
+            status = "peer failed"
+        q.put((rank, status, (addrs, own, pg.bufs.part_offsets), released))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("fail_rank", [-1, 0])
+def test_peer_group_maps_every_other_rank_and_releases_once(fail_rank):
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_group_worker, args=(r, world, port, q, fail_rank)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    try:
+        for _ in range(world):
+            r = q.get(timeout=120)
+            res[r[0]] = r[1:]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+    for rank in range(world):
+        status, payload, released = res[rank]
+        if rank == fail_rank:
+            # the import of the last rank failed: the one made before it is released, then the error surfaces
+            assert status == "raised" and "refused" in payload
+            others = [s for s in range(world) if s not in (rank, world - 1)]
+            assert released == [((1 << 40) * (s + 1), f"handle-{s}".encode()) for s in others]
+            continue
+        assert status == ("ok" if fail_rank < 0 else "peer failed")
+        (x_grp, sums), own, offs = payload
+        for s in range(world):
+            base = own[0] - offs[0] if s == rank else (1 << 40) * (s + 1)
+            assert x_grp[s] == base + offs[0] and sums[s] == base + offs[3]
+        assert sorted(released) == sorted(((1 << 40) * (s + 1), f"handle-{s}".encode())
+                                          for s in range(world) if s != rank)
